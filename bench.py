@@ -1,0 +1,456 @@
+"""Benchmark of the MoE layer with zero-computation experts (forward + expert-bias update) on B200.
+
+One step = lc_moe_forward on one batch (router GEMM, softmax + biased top-K + histogram, grouping,
+row gather, grouped SwiGLU GEMM, grouped down GEMM, combine) followed by the expert-bias update
+(with an all-reduce of the 768 expert counts when several ranks run). Default workload: the
+LongCat-Flash-shape prefill batch (T=16384 tokens per GPU, d=6144, 512 FFN experts of width 2048,
+256 zero experts, K=12, K_e=8, Zipf(1.1) expert popularity), synthetic data.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). ``--impl reference`` times the CPU oracle (test infrastructure) on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import pathlib
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = pathlib.Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "MoE-layer tokens/sec on 1 B200; grouped-GEMM % BF16 TC peak; permute/combine HBM GB/s"
+UNIT = "tokens/s"
+# the stages of lc_moe_forward, in launch order; kernels per stage
+STAGES = ("router_gemm", "topk", "permute", "gather", "gemm1_swiglu", "gemm2_down", "combine")
+KERNELS_PER_STAGE = (1, 1, 3, 1, 1, 1, 1)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clock sampler --
+
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu=timestamp,{self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for r in csv.reader(io.StringIO(pathlib.Path(self.path).read_text())):
+            r = [c.strip() for c in r]
+            if len(r) < 10:
+                continue
+            if self.uuid and self.uuid not in r[1]:
+                continue
+            rows.append(r)
+        os.unlink(self.path)
+        return rows
+
+    @staticmethod
+    def summarize(rows, window=None):
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return float("nan")
+        power = np.array([num(r[4]) for r in rows])
+        sm = np.array([num(r[2]) for r in rows])
+        loaded = power > 0.5 * np.nanmax(power) if np.isfinite(power).any() else np.ones(len(rows), bool)
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": float(np.nanmedian(sm[loaded])) if loaded.any() else float(np.nanmedian(sm)),
+                "sm_max_mhz": float(np.nanmax([num(r[3]) for r in rows])),
+                "reasons": sorted(reasons), "samples": int(len(rows)),
+                "samples_under_load": int(loaded.sum())}
+
+
+# ------------------------------------------------------------------------------- our arm ----
+
+def traffic_record(peaks_kernel: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if it was taken
+    on the current kernel source."""
+    p = ROOT / "profiles" / "traffic.json"
+    if not p.exists():
+        return None
+    rec = json.loads(p.read_text()).get(peaks_kernel)
+    if not rec:
+        return None
+    src = ROOT / "mixture_experts_zero_b200" / "csrc" / rec["source"]
+    if not src.exists() or hashlib.sha256(src.read_bytes()).hexdigest()[:16] != rec["sha256_16"]:
+        return None
+    return rec
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from mixture_experts_zero_b200 import binding as B
+    from mixture_experts_zero_b200 import inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    w = inputs.WORKLOADS[args.workload]
+    # weights identical on every rank (same seed); each rank draws its own tokens
+    data = inputs.make(w, device=dev, grid=False, experts=True)
+    if rank > 0:
+        g = inputs.generator(w.seed * 1000 + rank, dev)
+        data["x"] = inputs.draw_x(w, g, dev)
+    x, wr, bias, w13, w2 = data["x"], data["wr"], data["bias"], data["w13"], data["w2"]
+    bias = bias.clone()
+    T, E, K = w.T, w.E, w.K
+    shape = B.Shape(T, w.d, w.N, w.Z, K, w.I)
+    ws = B.new_workspace(shape, B.OP_FORWARD, dev)
+    out = torch.empty(T, w.d, dtype=torch.bfloat16, device=dev)
+    counts = torch.zeros(E, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    T_all = T * world
+
+    def step(events=None, xin=x, o=out):
+        B.lc_moe_forward(xin, wr, bias, w13, w2, K, out=o, counts=counts, ws=ws, stream=stream,
+                         events=events)
+        if world > 1:
+            dist.all_reduce(counts)
+        B.lc_moe_bias_update(bias, counts, T_all, w.N, w.Z, K, w.K_e, w.mu, reset_counts=True,
+                             stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(dev)
+
+    # ---- device-resident timing
+    for _ in range(args.warmup):
+        step()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    for row in ev:  # create the events before the timed region
+        for e in row:
+            e.record(stream)
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(events=ev[i])
+    t_end.record(stream)
+    barrier()
+    clock_rows = sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    stage_ms = np.array([[row[j].elapsed_time(row[j + 1]) for j in range(len(STAGES))] for row in ev])
+    if B.lc_moe_read_status(ws, stream=stream, raise_on_error=False):
+        raise SystemExit("device status bits set during the benchmark")
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    value = T * world * args.steps / (elapsed_ms / 1e3)
+
+    # routing statistics of this batch (one more untimed pass, counts not reset)
+    counts.zero_()
+    B.lc_moe_forward(x, wr, bias, w13, w2, K, out=out, counts=counts, ws=ws, stream=stream)
+    c = counts.cpu().numpy().astype(np.int64)
+    M = int(c[: w.N].sum())
+    touched = int((c[: w.N] > 0).sum())
+
+    # ---- end to end through the public API: pinned host x -> device, layer, out -> pinned host
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty(T, w.d, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(max(1, args.warmup // 2)):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(xin=x_dev)
+        out_host.copy_(out, non_blocking=True)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 20))
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(xin=x_dev)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t.item())
+    e2e_value = T * world * e2e_steps / (e2e_ms / 1e3)
+
+    # ---- roofline of each stage (algorithmic work only)
+    peaks, peak_src = load_peaks()
+    d_, I_ = w.d, w.I
+    wbytes_touched = touched * 3 * d_ * I_ * 2
+    alg = {
+        "router_gemm": ("tensor", 2.0 * T * d_ * E),
+        "topk": ("hbm", T * E * 4 + T * K * 8 + E * 4),
+        "permute": ("hbm", 2 * T * K * 4 + M * 4 + T * K * 4),
+        "gather": ("hbm", T * d_ * 2 + M * d_ * 2),
+        "gemm1_swiglu": ("tensor", 4.0 * M * d_ * I_),
+        "gemm2_down": ("tensor", 2.0 * M * d_ * I_),
+        "combine": ("hbm", M * d_ * 2 + 2 * T * d_ * 2 + T * K * 8),
+    }
+    med = np.median(stage_ms, axis=0)
+    mean = np.mean(stage_ms, axis=0)
+    stages = {}
+    for j, name in enumerate(STAGES):
+        bound, work = alg[name]
+        t_s = mean[j] / 1e3
+        if bound == "tensor":
+            ach = work / t_s / 1e12
+            peak = peaks["bf16_tflops_sustained"]
+            unit = "TFLOP/s"
+        else:
+            ach = work / t_s / 1e9
+            peak = peaks["hbm_gbs"]
+            unit = "GB/s"
+        stages[name] = {"ms": round(float(mean[j]), 4), "ms_median": round(float(med[j]), 4),
+                        "share": round(float(mean[j] / mean.sum()), 4), "bound": bound,
+                        "achieved": round(ach, 2), "unit": unit, "peak": peak,
+                        "frac": round(ach / peak, 4), "algorithmic_work": work}
+    dom = max(STAGES, key=lambda n: stages[n]["ms"])
+    ds = stages[dom]
+    trec = traffic_record(dom)
+    roofline = {"bound": ds["bound"], "kernel": dom, "achieved": ds["achieved"], "peak": ds["peak"],
+                "unit": ds["unit"], "frac": ds["frac"],
+                "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if ds['bound'] == 'tensor' else 'hbm_gbs'}, MEASURED_PEAKS.json)"
+                if peak_src == "measured" else "fallback",
+                "traffic": (trec["dram_bytes_per_launch"] if trec else None),
+                "algorithmic_per_launch": ds["algorithmic_work"]}
+    # whole-step roofline: max(FLOP / sustained TC peak, touched weights + activations / HBM)
+    flops = 2.0 * T * d_ * E + 6.0 * M * d_ * I_
+    bytes_ = wbytes_touched + E * d_ * 2 + 2 * T * d_ * 2
+    t_roof = max(flops / (peaks["bf16_tflops_sustained"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9))
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random-init weights of the LongCat-Flash MoE-layer shape)",
+        "config": {"workload": f"{w.name}: LongCat-Flash-shape MoE layer, prefill batch per GPU",
+                   "T": T, "d": d_, "N": w.N, "Z": w.Z, "K": K, "K_e": w.K_e, "I": I_,
+                   "router": w.router, "mu": w.mu, "parallelism": f"dp{world}",
+                   "step": "forward + counts all-reduce (N>1) + expert-bias update",
+                   "l2": "inputs larger than L2 (38.6 GB expert weights, 201 MB x per step)"},
+        "roofline": roofline,
+        "layer_roofline": {"t_roof_ms": round(t_roof * 1e3, 4), "frac": round(t_roof * 1e3 / ms_per_step, 4),
+                           "alg_flop": flops, "alg_bytes": bytes_, "ffn_rows_M": M,
+                           "experts_touched": touched,
+                           "zero_expert_share": round(float(c[w.N:].sum()) / (T * K), 4),
+                           "ffn_per_token": round(M / T, 4)},
+        "stages": stages,
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": int(x.numel() * 2),
+                "d2h_bytes_per_step": int(out.numel() * 2), "steps": e2e_steps},
+        "gpu_launches": int(args.steps * (sum(KERNELS_PER_STAGE) + 1)),
+        "clocks": ClockSampler.summarize(clock_rows),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, data, budget_s=args.cpu_budget)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ------------------------------------------------------------------- oracle (CPU baseline) ---
+
+def oracle_sample_step(w, x_bits, wr_bits, bias, expert_fetch, tokens):
+    """Run the oracle on ``tokens`` of the batch; return (seconds of oracle compute, n tokens)."""
+    import oracle
+    t0 = time.perf_counter()
+    xs = np.ascontiguousarray(x_bits[tokens])
+    z = oracle.router_logits(xs, wr_bits)
+    idx, gate, _, _ = oracle.route(z, bias, w.K)
+    t_oracle = time.perf_counter() - t0
+    pairs = [(i, r) for i in range(len(tokens)) for r in range(w.K) if idx[i, r] < w.N]
+    Y = np.empty((len(pairs), w.d), np.uint16)
+    pr = np.full((len(tokens), w.K), -1, np.int32)
+    experts = np.array([idx[i, r] for i, r in pairs], np.int64)
+    for e in np.unique(experts):
+        sel = np.nonzero(experts == e)[0]
+        w13e, w2e = expert_fetch(int(e))           # host copy, not timed
+        rows = np.ascontiguousarray(xs[[pairs[j][0] for j in sel]])
+        t0 = time.perf_counter()
+        _, y = oracle.expert_rows(rows, np.zeros(sel.size, np.int32), w13e, w2e, want_h=False)
+        t_oracle += time.perf_counter() - t0
+        Y[sel] = y
+    for j, (i, r) in enumerate(pairs):
+        pr[i, r] = j
+    t0 = time.perf_counter()
+    oracle.combine(xs, Y, idx, gate, pr, w.N)
+    t_oracle += time.perf_counter() - t0
+    return t_oracle, len(tokens)
+
+
+def cpu_baseline(w, data, budget_s: float = 20.0):
+    import oracle
+    from mixture_experts_zero_b200 import inputs
+    x_bits = inputs.bits(data["x"])
+    wr_bits = inputs.bits(data["wr"])
+    bias = data["bias"].cpu().numpy()
+
+    def fetch(e):
+        return (inputs.bits(data["w13"][e]).reshape(1, 2 * w.I, w.d),
+                inputs.bits(data["w2"][e]).reshape(1, w.d, w.I))
+
+    rng = np.random.default_rng(123)
+    n = 4
+    spent = tok = 0.0
+    while spent < budget_s:
+        tokens = np.sort(rng.choice(w.T, n, replace=False))
+        s, k = oracle_sample_step(w, x_bits, wr_bits, bias, fetch, tokens)
+        spent += s
+        tok += k
+        if spent < budget_s / 4:
+            n = min(n * 2, 64)
+    return {"value": round(tok / spent, 3), "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{int(tok)} random tokens of the {w.name} batch (router logits, routing, "
+                      f"SwiGLU experts of their FFN picks, combine), {spent:.1f} s of oracle time; "
+                      "expert weights copied to the host per expert outside the timed calls"}
+
+
+# --------------------------------------------------------------------------- reference arm --
+
+def run_reference(args):
+    """The oracle (CPU, plain C) as the reference arm, on bounded samples of the same workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+    import oracle
+    from mixture_experts_zero_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    g = inputs.generator(w.seed, "cpu")
+    wr_bits = inputs.bits(inputs.draw_router(w, g, "cpu"))
+    bias = inputs.draw_bias(w, g, "cpu").numpy()
+    cache = {}
+    std = 1.0 / math.sqrt(w.d)
+
+    def fetch(e):
+        if e not in cache:
+            ge = inputs.generator(w.seed * 100003 + e, "cpu")
+            w13 = (torch.randn(1, 2 * w.I, w.d, generator=ge) * std).to(torch.bfloat16)
+            w2 = (torch.randn(1, w.d, w.I, generator=ge) * std).to(torch.bfloat16)
+            cache[e] = (inputs.bits(w13), inputs.bits(w2))
+        return cache[e]
+
+    per_step_tokens = args.ref_tokens
+    total_s = total_tok = 0.0
+    for i in range(args.warmup + args.steps):
+        gx = inputs.generator(w.seed * 7919 + i, "cpu")
+        xs = torch.randn(per_step_tokens, w.d, generator=gx)
+        if w.router == "zipf":
+            xs[:, 0] = 1.0
+        x_bits = inputs.bits(xs.to(torch.bfloat16))
+        s, k = oracle_sample_step(w, x_bits, wr_bits, bias, fetch, np.arange(per_step_tokens))
+        if i >= args.warmup:
+            total_s += s
+            total_tok += k
+    value = total_tok / total_s
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_s / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: LongCat-Flash-shape MoE layer, prefill batch", "T": w.T,
+                   "d": w.d, "N": w.N, "Z": w.Z, "K": w.K, "K_e": w.K_e, "I": w.I,
+                   "router": w.router, "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{per_step_tokens} fresh tokens per step of the {w.name} workload"},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill", choices=["prefill", "decode", "small", "tiny"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time")
+    ap.add_argument("--ref-tokens", type=int, default=4, help="tokens per reference-arm step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,240 @@
+// common.cuh -- device helpers and internal launcher declarations of libmoezero.
+//
+// sm_100a only: mbarriers, TMA bulk-tensor loads, tcgen05 (5th-generation tensor core) MMA with
+// TMEM accumulators, written as inline PTX. No CUTLASS/CuTe code is used.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/lc_moe.h"
+
+namespace lcmoe {
+
+// ------------------------------------------------------------------------------ small utils --
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
+    if (status) atomicOr(status, bits);
+}
+
+// ---------------------------------------------------------------------------------- mbarrier --
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with parity `parity` of `bar`. Gives up (returns false) when the
+// CTA-wide abort flag is raised by another role, or after `limit_ns`, in which case it raises the
+// abort flag itself and records LC_MOE_DEV_WAIT_TIMEOUT.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                          volatile int* abort_flag, uint32_t* status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            set_status(status, LC_MOE_DEV_WAIT_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------- TMA --
+
+// 2-D tiled bulk-tensor load global -> shared, completion counted on `bar` (no multicast).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c0, int32_t c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ----------------------------------------------------------------------------------- tcgen05 --
+
+// TMEM allocation: whole warp, result (lane 0 / base column) written to shared memory.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand tile stored with the 128-byte swizzle:
+// rows of 64 bf16 (128 B), 8-row swizzle atoms of 1024 B stacked contiguously (stride-dimension
+// byte offset 1024). The leading-dimension offset is unused for swizzled K-major layouts.
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);  // start address >> 4, bits [0,14)
+    d |= static_cast<uint64_t>(1u) << 16;                 // leading byte offset (16 B) >> 4
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;         // stride byte offset >> 4
+    d |= static_cast<uint64_t>(1u) << 46;                 // descriptor version (sm_100)
+    d |= static_cast<uint64_t>(2u) << 61;                 // swizzle mode: 128 B
+    return d;
+}
+
+// Instruction descriptor, kind::f16: A and B bf16, K-major; D fp32; shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+    return (1u << 4)                                   // D format: f32
+           | (1u << 7)                                 // A format: bf16
+           | (1u << 10)                                // B format: bf16
+           | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, one 128 x N x 16 step, issued by a single thread.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "setp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
+        "}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05 operation issued so far by this thread has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives lane (base + i).
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------ bf16 pack helpers --
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ------------------------------------------------------------- internal launchers (host side) --
+
+struct DevInfo {
+    int sm_count;
+    int ok_sm100;
+};
+// Per-device cached properties of the current device (returns nullptr on a CUDA error).
+const DevInfo* current_device_info();
+
+uint64_t wait_limit_ns();
+
+// Router GEMM: logits[T, E] fp32 = x[T, d] * wr[E, d]^T.
+cudaError_t launch_router_gemm(const void* x, const void* wr, float* logits, int T, int d, int E,
+                               uint32_t* status, cudaStream_t st);
+
+// Grouped GEMM 1: h[rows, I] = silu(X Wg^T) * (X Wu^T) per expert group (rows from offsets).
+cudaError_t launch_grouped_swiglu(const void* x_perm, int64_t rows_cap, const int32_t* offsets,
+                                  int N, const void* w13, int d, int I, void* h, uint32_t* status,
+                                  cudaStream_t st);
+
+// Grouped GEMM 2: y[rows, d] = h Wd^T per expert group.
+cudaError_t launch_grouped_down(const void* h, int64_t rows_cap, const int32_t* offsets, int N,
+                                const void* w2, int d, int I, void* y, uint32_t* status,
+                                cudaStream_t st);
+
+cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int K, int32_t* idx,
+                        float* gate, int32_t* counts, uint32_t* status, cudaStream_t st);
+
+cudaError_t launch_hist(const int32_t* idx, int64_t n, int n_bins, int32_t* counts,
+                        uint32_t* status, cudaStream_t st);
+
+cudaError_t launch_bias_update(float* bias, int32_t* counts, int E, int64_t T_all, int N, int K,
+                               int K_e, float mu, int reset, cudaStream_t st);
+
+// Scratch of the grouping step: two [nblk, N] int32 tables.
+size_t permute_scratch_bytes(int T, int N);
+cudaError_t launch_permute(const int32_t* idx, int T, int K, int N, int E, int32_t* offsets,
+                           int32_t* row_token, int32_t* pair_row, int32_t* scratch,
+                           uint32_t* status, cudaStream_t st);
+cudaError_t launch_gather(const void* x, int T, int d, int K, const int32_t* pair_row,
+                          void* x_perm, cudaStream_t st);
+
+cudaError_t launch_combine(const void* x, const void* y, const float* gate,
+                           const int32_t* pair_row, int T, int d, int K, void* out,
+                           cudaStream_t st);
+
+}  // namespace lcmoe

@@ -1,0 +1,233 @@
+// permute.cu -- grouping of the (token, pick) pairs routed to FFN experts, and the row gather.
+//
+// Only the N FFN experts of the MoE equation (LongCat-Flash llm-wiki entity page, section 2.1)
+// do work; picks of the Z zero-computation experts (ids >= N) get no row, so they are never
+// copied, multiplied or written back (the combine adds their g x_t term directly).
+//
+// Deterministic stable counting sort, no atomics on positions:
+//   count   : block b owns tokens [256 b, 256 b + 256). For each FFN expert e it builds a 256-bit
+//             mask of the block's tokens that picked e (atomicOr in shared memory: order-free),
+//             and writes the block count popc(mask) to cnt[b][e].
+//   scan    : one block; for each expert a running sum over blocks gives base[b][e] (rows of e in
+//             earlier blocks), then an exclusive scan over experts gives offsets[e].
+//   scatter : the row of pick (t, r) of expert e is
+//             offsets[e] + base[b][e] + popc(mask of e restricted to tokens before t in block b),
+//             so rows of an expert are in ascending token order. Writes pair_row and row_token.
+//   gather  : one warp per token copies x_t (16-byte vectors) to each of its FFN rows; x_t is
+//             read once however many FFN experts the token picked.
+#include "common.cuh"
+
+namespace lcmoe {
+
+namespace {
+
+constexpr int PB = 256;          // tokens per block = threads per block
+constexpr int MASK_WORDS = PB / 32;
+
+__device__ __forceinline__ bool build_masks(const int32_t* __restrict__ idx, int T, int K, int N,
+                                            int E, uint32_t* mask, uint32_t* status) {
+    const int t = blockIdx.x * PB + threadIdx.x;
+    bool bad = false;
+    if (t < T) {
+        const uint32_t bit = 1u << (threadIdx.x & 31);
+        const int w = threadIdx.x >> 5;
+        for (int r = 0; r < K; ++r) {
+            const int e = idx[static_cast<int64_t>(t) * K + r];
+            if (e < 0 || e >= E) {
+                bad = true;
+            } else if (e < N) {
+                const uint32_t old = atomicOr(&mask[e * MASK_WORDS + w], bit);
+                if (old & bit) set_status(status, LC_MOE_DEV_DUP_PICK);
+            }
+        }
+    }
+    return bad;
+}
+
+__global__ void __launch_bounds__(PB)
+    perm_count_kernel(const int32_t* __restrict__ idx, int T, int K, int N, int E,
+                      int32_t* __restrict__ cnt, uint32_t* __restrict__ status) {
+    extern __shared__ uint32_t mask[];
+    for (int i = threadIdx.x; i < N * MASK_WORDS; i += PB) mask[i] = 0;
+    __syncthreads();
+    const bool bad = build_masks(idx, T, K, N, E, mask, status);
+    if (__syncthreads_or(bad) && threadIdx.x == 0) set_status(status, LC_MOE_DEV_IDX_RANGE);
+    for (int e = threadIdx.x; e < N; e += PB) {
+        int c = 0;
+#pragma unroll
+        for (int w = 0; w < MASK_WORDS; ++w) c += __popc(mask[e * MASK_WORDS + w]);
+        cnt[static_cast<int64_t>(blockIdx.x) * N + e] = c;
+    }
+}
+
+constexpr int SCAN_THREADS = 1024;
+
+__global__ void __launch_bounds__(SCAN_THREADS)
+    perm_scan_kernel(const int32_t* __restrict__ cnt, int nblk, int N, int32_t* __restrict__ base,
+                     int32_t* __restrict__ offsets) {
+    extern __shared__ int32_t tot[];  // [N]
+    __shared__ int32_t warp_sums[SCAN_THREADS / 32];
+    __shared__ int32_t carry;
+    for (int e = threadIdx.x; e < N; e += SCAN_THREADS) {
+        int run = 0;
+        int b = 0;
+        for (; b + 4 <= nblk; b += 4) {
+            const int c0 = cnt[static_cast<int64_t>(b) * N + e];
+            const int c1 = cnt[static_cast<int64_t>(b + 1) * N + e];
+            const int c2 = cnt[static_cast<int64_t>(b + 2) * N + e];
+            const int c3 = cnt[static_cast<int64_t>(b + 3) * N + e];
+            base[static_cast<int64_t>(b) * N + e] = run;
+            base[static_cast<int64_t>(b + 1) * N + e] = run + c0;
+            base[static_cast<int64_t>(b + 2) * N + e] = run + c0 + c1;
+            base[static_cast<int64_t>(b + 3) * N + e] = run + c0 + c1 + c2;
+            run += c0 + c1 + c2 + c3;
+        }
+        for (; b < nblk; ++b) {
+            const int c = cnt[static_cast<int64_t>(b) * N + e];
+            base[static_cast<int64_t>(b) * N + e] = run;
+            run += c;
+        }
+        tot[e] = run;
+    }
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    // exclusive scan of tot[0..N) in chunks of SCAN_THREADS
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int base_e = 0; base_e < N; base_e += SCAN_THREADS) {
+        const int e = base_e + threadIdx.x;
+        const int v = (e < N) ? tot[e] : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+        }
+        if (lane == 31) warp_sums[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            int ws = warp_sums[lane];
+            int wi = ws;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, wi, o);
+                if (lane >= o) wi += u;
+            }
+            warp_sums[lane] = wi - ws;  // exclusive prefix of warp totals
+        }
+        __syncthreads();
+        const int excl = carry + warp_sums[warp] + incl - v;
+        if (e < N) offsets[e] = excl;
+        __syncthreads();
+        if (threadIdx.x == SCAN_THREADS - 1) carry = excl + v;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) offsets[N] = carry;
+}
+
+__global__ void __launch_bounds__(PB)
+    perm_scatter_kernel(const int32_t* __restrict__ idx, int T, int K, int N, int E,
+                        const int32_t* __restrict__ base, const int32_t* __restrict__ offsets,
+                        int32_t* __restrict__ row_token, int32_t* __restrict__ pair_row) {
+    extern __shared__ uint32_t mask[];
+    for (int i = threadIdx.x; i < N * MASK_WORDS; i += PB) mask[i] = 0;
+    __syncthreads();
+    build_masks(idx, T, K, N, E, mask, nullptr);
+    __syncthreads();
+    const int t = blockIdx.x * PB + threadIdx.x;
+    if (t >= T) return;
+    const int w = threadIdx.x >> 5;
+    const uint32_t below = (1u << (threadIdx.x & 31)) - 1u;
+    for (int r = 0; r < K; ++r) {
+        const int e = idx[static_cast<int64_t>(t) * K + r];
+        int row = -1;
+        if (e >= 0 && e < N) {
+            int rank = __popc(mask[e * MASK_WORDS + w] & below);
+            for (int j = 0; j < w; ++j) rank += __popc(mask[e * MASK_WORDS + j]);
+            row = offsets[e] + base[static_cast<int64_t>(blockIdx.x) * N + e] + rank;
+            row_token[row] = t;
+        }
+        pair_row[static_cast<int64_t>(t) * K + r] = row;
+    }
+}
+
+constexpr int GATHER_THREADS = 256;
+
+__global__ void __launch_bounds__(GATHER_THREADS)
+    gather_kernel(const uint4* __restrict__ x, int T, int d8, int K, const int32_t* __restrict__ pair_row,
+                  uint4* __restrict__ x_perm) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warps_total = gridDim.x * (GATHER_THREADS / 32);
+    for (int t = blockIdx.x * (GATHER_THREADS / 32) + warp; t < T; t += warps_total) {
+        const int my_row = (lane < K) ? pair_row[static_cast<int64_t>(t) * K + lane] : -1;
+        const uint32_t dests = __ballot_sync(0xffffffffu, my_row >= 0);
+        if (!dests) continue;
+        const uint4* src = x + static_cast<int64_t>(t) * d8;
+        for (int c0 = 0; c0 < d8; c0 += 32) {  // warp-uniform trip count
+            const int c = c0 + lane;
+            const bool in = c < d8;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (in) v = __ldg(src + c);
+            uint32_t m = dests;
+            while (m) {
+                const int r = __ffs(m) - 1;
+                m &= m - 1;
+                const int row = __shfl_sync(0xffffffffu, my_row, r);
+                if (in) x_perm[static_cast<int64_t>(row) * d8 + c] = v;
+            }
+        }
+    }
+}
+
+}  // namespace
+
+size_t permute_scratch_bytes(int T, int N) {
+    const size_t nblk = (static_cast<size_t>(T) + PB - 1) / PB;
+    return 2 * nblk * static_cast<size_t>(N) * sizeof(int32_t);
+}
+
+cudaError_t launch_permute(const int32_t* idx, int T, int K, int N, int E, int32_t* offsets,
+                           int32_t* row_token, int32_t* pair_row, int32_t* scratch,
+                           uint32_t* status, cudaStream_t st) {
+    const int nblk = (T + PB - 1) / PB;
+    int32_t* cnt = scratch;
+    int32_t* base = scratch + static_cast<size_t>(nblk) * N;
+    const size_t mask_bytes = static_cast<size_t>(N) * MASK_WORDS * sizeof(uint32_t);
+    static bool configured[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && !configured[dev]) {
+        // masks of up to 2048 experts take 64 KB of shared memory
+        e = cudaFuncSetAttribute(perm_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2048 * MASK_WORDS * 4);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(perm_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2048 * MASK_WORDS * 4);
+        if (e != cudaSuccess) return e;
+        configured[dev] = true;
+    }
+    if (nblk > 0) {
+        perm_count_kernel<<<nblk, PB, mask_bytes, st>>>(idx, T, K, N, E, cnt, status);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    perm_scan_kernel<<<1, SCAN_THREADS, static_cast<size_t>(N) * sizeof(int32_t), st>>>(cnt, nblk, N, base, offsets);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (nblk > 0) {
+        perm_scatter_kernel<<<nblk, PB, mask_bytes, st>>>(idx, T, K, N, E, base, offsets, row_token, pair_row);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_gather(const void* x, int T, int d, int K, const int32_t* pair_row, void* x_perm,
+                          cudaStream_t st) {
+    const DevInfo* di = current_device_info();
+    if (!di) return cudaErrorUnknown;
+    if (T == 0) return cudaSuccess;
+    const int warps = GATHER_THREADS / 32;
+    int blocks = (T + warps - 1) / warps;
+    if (blocks > di->sm_count * 8) blocks = di->sm_count * 8;
+    gather_kernel<<<blocks, GATHER_THREADS, 0, st>>>(static_cast<const uint4*>(x), T, d / 8, K, pair_row,
+                                                      static_cast<uint4*>(x_perm));
+    return cudaGetLastError();
+}
+
+}  // namespace lcmoe

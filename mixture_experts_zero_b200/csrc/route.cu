@@ -1,0 +1,289 @@
+// route.cu -- routing of the MoE layer with zero-computation experts, and the expert-bias
+// controller (LongCat-Flash llm-wiki entity page, section 2.1; softmax gate: section 2.3.2).
+//
+//   topk      : per token, s = softmax(z) over all E = N + Z experts; key_i = s_i + b_i;
+//               the K largest keys in descending order (equal keys: lower index first);
+//               gate_r = s_sel[r] / (s_sel[0] + ... + s_sel[K-1]); optional histogram of picks.
+//   hist      : T_i, the number of picks of each expert (the T_i of the bias-update equation).
+//   bias      : b_i += mu * (K_e/(K N) - T_i/(K T_all)) for all E experts.
+//
+// Routing decisions are integers decided in fp32, so the fp32 steps are fixed exactly:
+//   exp: Cody-Waite reduction (Cody & Waite, Software Manual for the Elementary Functions, 1980)
+//        u = n ln2 + r, n = rint(u log2e), ln2 split into a 16-fraction-bit head and a tail,
+//        then e^r by its degree-7 Taylor polynomial (coefficients 1/k!) in Horner form with
+//        fused multiply-adds, times 2^n; inputs below -86 give 0;
+//   sum: lane l of the warp adds e_l, e_{l+32}, ... in order from +0, then the lanes combine by
+//        a butterfly over xor distances 16, 8, 4, 2, 1 (both operands of every add are the same
+//        pair of values on the two lanes, so all lanes end with identical bits);
+//   every other step is one IEEE round-to-nearest operation (__f*_rn intrinsics, no contraction).
+#include "common.cuh"
+
+namespace lcmoe {
+
+namespace {
+
+// fp32 constants of the exp above, from ln 2 and 1/k!
+__device__ __forceinline__ float exp_spec(float u) {
+    const float LOG2E = 0x1.715476p+0f;     // 1/ln 2, rounded to fp32
+    const float LN2_HI = 0x1.62e4p-1f;      // ln 2 rounded to 16 fraction bits (exact)
+    const float LN2_LO = 0x1.7f7d1cp-20f;   // ln 2 - LN2_HI, rounded to fp32
+    if (u != u) return u;
+    if (u < -86.0f) return 0.0f;
+    if (u > 88.0f) return __int_as_float(0x7f800000);
+    const float n = rintf(__fmul_rn(u, LOG2E));
+    float r = __fmaf_rn(-n, LN2_HI, u);
+    r = __fmaf_rn(-n, LN2_LO, r);
+    float p = 0x1.a01a02p-13f;              // 1/7!
+    p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);   // 1/6!
+    p = __fmaf_rn(p, r, 0x1.111112p-7f);    // 1/5!
+    p = __fmaf_rn(p, r, 0x1.555556p-5f);    // 1/4!
+    p = __fmaf_rn(p, r, 0x1.555556p-3f);    // 1/3!
+    p = __fmaf_rn(p, r, 0.5f);              // 1/2!
+    p = __fmaf_rn(p, r, 1.0f);              // 1/1!
+    p = __fmaf_rn(p, r, 1.0f);              // 1/0!
+    const float scale = __int_as_float((static_cast<int>(n) + 127) << 23);  // 2^n, normal
+    return __fmul_rn(p, scale);
+}
+
+// (key, index) order of the selection: larger key first, equal keys lower index first.
+__device__ __forceinline__ bool better(float ka, int ia, float kb, int ib) {
+    if (ib < 0) return ia >= 0;
+    if (ia < 0) return false;
+    return ka > kb || (ka == kb && ia < ib);
+}
+
+constexpr int TOPK_THREADS = 256;  // 8 warps, one token per warp at a time
+
+template <int VPL>
+__global__ void __launch_bounds__(TOPK_THREADS)
+    topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
+                int K, int32_t* __restrict__ idx, float* __restrict__ gate,
+                int32_t* __restrict__ counts, uint32_t* __restrict__ status) {
+    extern __shared__ int32_t s_hist[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const bool do_hist = counts != nullptr;
+    if (do_hist)
+        for (int i = threadIdx.x; i < E; i += TOPK_THREADS) s_hist[i] = 0;
+    __syncthreads();
+
+    float b[VPL];
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        const int i = lane + 32 * j;
+        b[j] = (i < E) ? bias[i] : 0.0f;
+    }
+
+    const int warps_total = gridDim.x * (TOPK_THREADS / 32);
+    for (int t = blockIdx.x * (TOPK_THREADS / 32) + warp; t < T; t += warps_total) {
+        const float* zt = logits + static_cast<int64_t>(t) * E;
+        float v[VPL];
+        float m = __int_as_float(0xff800000);  // -inf
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            const int i = lane + 32 * j;
+            v[j] = (i < E) ? zt[i] : __int_as_float(0xff800000);
+            m = (v[j] > m) ? v[j] : m;  // a NaN logit is skipped here, and poisons the sum below
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const float other = __shfl_xor_sync(0xffffffffu, m, o);
+            m = (other > m) ? other : m;
+        }
+        // e_i = EXP(z_i - m); lane partial sums in index order
+        float part = 0.0f;
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            const int i = lane + 32 * j;
+            if (i < E) {
+                v[j] = exp_spec(__fsub_rn(v[j], m));
+                part = __fadd_rn(part, v[j]);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
+        const float S = part;
+        // scores s_i and keys s_i + b_i
+        float key[VPL];
+        bool nan_key = false;
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            const int i = lane + 32 * j;
+            if (i < E) {
+                v[j] = __fdiv_rn(v[j], S);
+                key[j] = __fadd_rn(v[j], b[j]);
+                nan_key |= (key[j] != key[j]);
+            }
+        }
+        if (__any_sync(0xffffffffu, nan_key)) {
+            if (lane == 0) set_status(status, LC_MOE_DEV_NAN_KEY);
+            if (lane < K) {
+                idx[static_cast<int64_t>(t) * K + lane] = lane;
+                gate[static_cast<int64_t>(t) * K + lane] = __int_as_float(0x7fc00000);
+                if (do_hist) atomicAdd(&s_hist[lane], 1);
+            }
+            continue;
+        }
+        // K rounds of warp arg-max over (key, index)
+        uint64_t taken = 0;
+        float lk = 0.0f, ls = 0.0f;
+        int li = -1;
+        auto local_best = [&]() {
+            li = -1;
+#pragma unroll
+            for (int j = 0; j < VPL; ++j) {
+                const int i = lane + 32 * j;
+                if (i < E && !((taken >> j) & 1ull) && (li < 0 || key[j] > lk)) {
+                    lk = key[j];
+                    ls = v[j];
+                    li = i;
+                }
+            }
+        };
+        local_best();
+        int my_idx = 0;
+        float my_s = 0.0f;
+        for (int r = 0; r < K; ++r) {
+            float bk = lk, bs = ls;
+            int bi = li;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+                const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (better(ok, oi, bk, bi)) {
+                    bk = ok;
+                    bs = os;
+                    bi = oi;
+                }
+            }
+            if (lane == r) {
+                my_idx = bi;
+                my_s = bs;
+            }
+            if (bi >= 0 && (bi & 31) == lane) {
+                taken |= 1ull << (bi >> 5);
+                local_best();
+            }
+        }
+        // renormalise over the K chosen, summing in rank order
+        float Q = 0.0f;
+        for (int r = 0; r < K; ++r) Q = __fadd_rn(Q, __shfl_sync(0xffffffffu, my_s, r));
+        if (lane < K) {
+            idx[static_cast<int64_t>(t) * K + lane] = my_idx;
+            gate[static_cast<int64_t>(t) * K + lane] = __fdiv_rn(my_s, Q);
+            if (do_hist) atomicAdd(&s_hist[my_idx], 1);
+        }
+    }
+    if (do_hist) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < E; i += TOPK_THREADS) {
+            const int c = s_hist[i];
+            if (c) atomicAdd(&counts[i], c);
+        }
+    }
+}
+
+template <int VPL>
+cudaError_t launch_topk_t(const float* logits, const float* bias, int T, int E, int K,
+                          int32_t* idx, float* gate, int32_t* counts, uint32_t* status,
+                          cudaStream_t st, int sm_count) {
+    const int warps = TOPK_THREADS / 32;
+    int blocks = (T + warps - 1) / warps;
+    const int cap = sm_count * 4;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    const size_t smem = counts ? static_cast<size_t>(E) * sizeof(int32_t) : 0;
+    topk_kernel<VPL><<<blocks, TOPK_THREADS, smem, st>>>(logits, bias, T, E, K, idx, gate, counts,
+                                                          status);
+    return cudaGetLastError();
+}
+
+constexpr int HIST_THREADS = 512;
+
+__global__ void __launch_bounds__(HIST_THREADS)
+    hist_kernel(const int32_t* __restrict__ idx, int64_t n, int n_bins, int32_t* __restrict__ counts,
+                uint32_t* __restrict__ status) {
+    extern __shared__ int32_t s_hist[];
+    for (int i = threadIdx.x; i < n_bins; i += HIST_THREADS) s_hist[i] = 0;
+    __syncthreads();
+    bool bad = false;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * HIST_THREADS;
+    const int64_t n4 = n / 4;
+    const int4* idx4 = reinterpret_cast<const int4*>(idx);
+    for (int64_t p = static_cast<int64_t>(blockIdx.x) * HIST_THREADS + threadIdx.x; p < n4; p += stride) {
+        const int4 q = __ldg(idx4 + p);
+        const int vals[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (vals[j] >= 0 && vals[j] < n_bins) atomicAdd(&s_hist[vals[j]], 1);
+            else bad = true;
+        }
+    }
+    for (int64_t p = n4 * 4 + static_cast<int64_t>(blockIdx.x) * HIST_THREADS + threadIdx.x; p < n; p += stride) {
+        const int v = idx[p];
+        if (v >= 0 && v < n_bins) atomicAdd(&s_hist[v], 1);
+        else bad = true;
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) set_status(status, LC_MOE_DEV_IDX_RANGE);
+    for (int i = threadIdx.x; i < n_bins; i += HIST_THREADS) {
+        const int c = s_hist[i];
+        if (c) atomicAdd(&counts[i], c);
+    }
+}
+
+__global__ void bias_update_kernel(float* __restrict__ bias, int32_t* __restrict__ counts, int E,
+                                   long long T_all, int N, int K, int K_e, float mu, int reset) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= E) return;
+    const float kn = __fmul_rn(static_cast<float>(K), static_cast<float>(N));
+    const float a = __fdiv_rn(static_cast<float>(K_e), kn);
+    const float kt = __fmul_rn(static_cast<float>(K), __ll2float_rn(T_all));
+    const float c = __fdiv_rn(__int2float_rn(counts[i]), kt);
+    const float delta = __fmul_rn(mu, __fsub_rn(a, c));
+    bias[i] = __fadd_rn(bias[i], delta);
+    if (reset) counts[i] = 0;
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const float* logits, const float* bias, int T, int E, int K, int32_t* idx,
+                        float* gate, int32_t* counts, uint32_t* status, cudaStream_t st) {
+    const DevInfo* di = current_device_info();
+    if (!di) return cudaErrorUnknown;
+    const int vpl = (E + 31) / 32;
+    const int sm = di->sm_count;
+    if (vpl <= 1) return launch_topk_t<1>(logits, bias, T, E, K, idx, gate, counts, status, st, sm);
+    if (vpl <= 2) return launch_topk_t<2>(logits, bias, T, E, K, idx, gate, counts, status, st, sm);
+    if (vpl <= 4) return launch_topk_t<4>(logits, bias, T, E, K, idx, gate, counts, status, st, sm);
+    if (vpl <= 8) return launch_topk_t<8>(logits, bias, T, E, K, idx, gate, counts, status, st, sm);
+    if (vpl <= 12) return launch_topk_t<12>(logits, bias, T, E, K, idx, gate, counts, status, st, sm);
+    if (vpl <= 16) return launch_topk_t<16>(logits, bias, T, E, K, idx, gate, counts, status, st, sm);
+    if (vpl <= 24) return launch_topk_t<24>(logits, bias, T, E, K, idx, gate, counts, status, st, sm);
+    if (vpl <= 32) return launch_topk_t<32>(logits, bias, T, E, K, idx, gate, counts, status, st, sm);
+    if (vpl <= 48) return launch_topk_t<48>(logits, bias, T, E, K, idx, gate, counts, status, st, sm);
+    return launch_topk_t<64>(logits, bias, T, E, K, idx, gate, counts, status, st, sm);
+}
+
+cudaError_t launch_hist(const int32_t* idx, int64_t n, int n_bins, int32_t* counts,
+                        uint32_t* status, cudaStream_t st) {
+    const DevInfo* di = current_device_info();
+    if (!di) return cudaErrorUnknown;
+    int64_t blocks = (n / 4 + HIST_THREADS - 1) / HIST_THREADS;
+    if (blocks > di->sm_count * 2) blocks = di->sm_count * 2;
+    if (blocks < 1) blocks = 1;
+    hist_kernel<<<static_cast<int>(blocks), HIST_THREADS, static_cast<size_t>(n_bins) * 4, st>>>(
+        idx, n, n_bins, counts, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bias_update(float* bias, int32_t* counts, int E, int64_t T_all, int N, int K,
+                               int K_e, float mu, int reset, cudaStream_t st) {
+    const int threads = 256;
+    const int blocks = (E + threads - 1) / threads;
+    bias_update_kernel<<<blocks, threads, 0, st>>>(bias, counts, E, static_cast<long long>(T_all), N,
+                                                   K, K_e, mu, reset);
+    return cudaGetLastError();
+}
+
+}  // namespace lcmoe

@@ -40,8 +40,9 @@ def configure(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_permute.argtypes = [P, I64, I64, I64, P, P, P]
     L.oracle_permute.restype = I64
     L.oracle_expert_rows.argtypes = [P, P, I64, I64, I64, P, P, P, P]
-    L.oracle_combine.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P]
-    L.oracle_forward.argtypes = [P, P, P, P, P, I64, I64, I64, I64, I64, I64, P, P, P, P, P]
+    L.oracle_expert_down.argtypes = [P, P, I64, I64, I64, P, P]
+    L.oracle_combine.argtypes = [P, P, P, P, P, I64, I64, I64, I64, P, P]
+    L.oracle_forward.argtypes = [P, P, P, P, P, I64, I64, I64, I64, I64, I64, P, P, P, P, P, P]
     L.oracle_forward.restype = I64
     L.oracle_bias_update.argtypes = [P, P, I64, I64, I64, I64, I64, ctypes.c_float]
     return L
@@ -161,20 +162,36 @@ def expert_rows(xrows: np.ndarray, row_expert: np.ndarray, w13: np.ndarray, w2: 
     return h, y
 
 
+def expert_down(h: np.ndarray, row_expert: np.ndarray, w2: np.ndarray) -> np.ndarray:
+    """The down projection alone: Y = bf16(H Wd[e]^T) for given bf16 rows H [M, I]."""
+    h = _c(h, np.uint16); row_expert = _c(row_expert, np.int32); w2 = _c(w2, np.uint16)
+    M, I = h.shape
+    n, d, I2 = w2.shape
+    assert I2 == I and row_expert.shape == (M,)
+    if M and (row_expert.min() < 0 or row_expert.max() >= n):
+        raise ValueError("row_expert out of range")
+    y = np.empty((M, d), dtype=np.uint16)
+    lib().oracle_expert_down(_p(h), _p(row_expert), M, d, I, _p(w2), _p(y))
+    return y
+
+
 def combine(x: np.ndarray, y: np.ndarray, idx: np.ndarray, gate: np.ndarray,
-            pair_row: np.ndarray, N: int) -> np.ndarray:
-    """out_t = bf16(sum_r g_r * (Y[pair_row] if FFN pick else x_t)), double, rank order."""
+            pair_row: np.ndarray, N: int, want_exact: bool = False):
+    """out_t = bf16(sum_r g_r * (Y[pair_row] if FFN pick else x_t)), double, rank order.
+    With ``want_exact`` returns (out, the double sums before rounding)."""
     x = _c(x, np.uint16); y = _c(y, np.uint16); idx = _c(idx, np.int32)
     gate = _c(gate, np.float32); pair_row = _c(pair_row, np.int32)
     T, d = x.shape
     K = idx.shape[1]
     out = np.empty((T, d), dtype=np.uint16)
-    lib().oracle_combine(_p(x), _p(y), _p(idx), _p(gate), _p(pair_row), T, d, K, N, _p(out))
-    return out
+    acc = np.empty((T, d), dtype=np.float64) if want_exact else None
+    lib().oracle_combine(_p(x), _p(y), _p(idx), _p(gate), _p(pair_row), T, d, K, N, _p(out), _p(acc))
+    return (out, acc) if want_exact else out
 
 
 def forward(x, wr, bias, w13, w2, N: int, Z: int, K: int, counts: np.ndarray | None = None):
-    """The whole layer from the MoE equation. Returns dict(out, logits, idx, gate, counts, bad)."""
+    """The whole layer from the MoE equation. Returns dict(out, out_exact, logits, idx, gate,
+    counts, bad); out_exact holds the double sums before their rounding to bf16."""
     x = _c(x, np.uint16); wr = _c(wr, np.uint16); bias = _c(bias, np.float32)
     w13 = _c(w13, np.uint16); w2 = _c(w2, np.uint16)
     T, d = x.shape
@@ -186,9 +203,10 @@ def forward(x, wr, bias, w13, w2, N: int, Z: int, K: int, counts: np.ndarray | N
     idx = np.empty((T, K), dtype=np.int32)
     gate = np.empty((T, K), dtype=np.float32)
     cnt = np.zeros(E, dtype=np.int32) if counts is None else _c(counts, np.int32)
+    acc = np.empty((T, d), dtype=np.float64)
     bad = lib().oracle_forward(_p(x), _p(wr), _p(bias), _p(w13), _p(w2), T, d, N, Z, K, I,
-                               _p(out), _p(logits), _p(idx), _p(gate), _p(cnt))
-    return dict(out=out, logits=logits, idx=idx, gate=gate, counts=cnt, bad=int(bad))
+                               _p(out), _p(logits), _p(idx), _p(gate), _p(cnt), _p(acc))
+    return dict(out=out, out_exact=acc, logits=logits, idx=idx, gate=gate, counts=cnt, bad=int(bad))
 
 
 def bias_update(bias: np.ndarray, counts: np.ndarray, T_all: int, N: int, Z: int, K: int,

@@ -259,6 +259,15 @@ int64_t oracle_permute(const int32_t* idx, int64_t T, int64_t K, int64_t N,
 /* row_expert 0.                                                                               */
 /* ------------------------------------------------------------------------------------------ */
 
+/* Down projection of one row: Y_i = bf16( sum_j H_j Wd[i][j] ), double accumulation. */
+static void down_row(const double* hd, const uint16_t* wd, int64_t d, int64_t I, uint16_t* yrow) {
+    for (int64_t i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int64_t j = 0; j < I; ++j) acc += hd[j] * bf16_to_double(wd[i * I + j]);
+        yrow[i] = oracle_double_to_bf16(acc);
+    }
+}
+
 void oracle_expert_rows(const uint16_t* xrows, const int32_t* row_expert, int64_t M, int64_t d,
                         int64_t I, const uint16_t* w13, const uint16_t* w2, uint16_t* h,
                         uint16_t* y) {
@@ -283,23 +292,32 @@ void oracle_expert_rows(const uint16_t* xrows, const int32_t* row_expert, int64_
             if (h) h[r * I + j] = hb;
             hd[j] = bf16_to_double(hb);
         }
-        for (int64_t i = 0; i < d; ++i) {
-            double acc = 0.0;
-            for (int64_t j = 0; j < I; ++j) acc += hd[j] * bf16_to_double(wd[i * I + j]);
-            y[r * d + i] = oracle_double_to_bf16(acc);
-        }
+        down_row(hd, wd, d, I, y + r * d);
         free(xd); free(hd);
+    }
+}
+
+/* The down projection alone, from given bf16 rows H [M, I]: Y = bf16(H Wd[e]^T). */
+void oracle_expert_down(const uint16_t* h, const int32_t* row_expert, int64_t M, int64_t d,
+                        int64_t I, const uint16_t* w2, uint16_t* y) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < M; ++r) {
+        double* hd = (double*)malloc((size_t)I * sizeof(double));
+        for (int64_t j = 0; j < I; ++j) hd[j] = bf16_to_double(h[r * I + j]);
+        down_row(hd, w2 + (int64_t)row_expert[r] * d * I, d, I, y + r * d);
+        free(hd);
     }
 }
 
 /* ------------------------------------------------------------------------------------------ */
 /* Step 8: combine. out_t = bf16( sum_r g_r * v_r ), v_r = Y[pair_row[t,r]] for an FFN pick    */
 /* and v_r = x_t for a zero-computation pick (E_i(x) = x), summed in double in rank order.     */
+/* out_acc (optional, [T, d]) receives the double sum before its rounding to bf16.             */
 /* ------------------------------------------------------------------------------------------ */
 
 void oracle_combine(const uint16_t* x, const uint16_t* y, const int32_t* idx, const float* gate,
                     const int32_t* pair_row, int64_t T, int64_t d, int64_t K, int64_t N,
-                    uint16_t* out) {
+                    uint16_t* out, double* out_acc) {
     #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; ++t) {
         for (int64_t c = 0; c < d; ++c) {
@@ -311,6 +329,7 @@ void oracle_combine(const uint16_t* x, const uint16_t* y, const int32_t* idx, co
                 acc += g * v;
             }
             out[t * d + c] = oracle_double_to_bf16(acc);
+            if (out_acc) out_acc[t * d + c] = acc;
         }
     }
 }
@@ -318,13 +337,14 @@ void oracle_combine(const uint16_t* x, const uint16_t* y, const int32_t* idx, co
 /* ------------------------------------------------------------------------------------------ */
 /* The whole layer, straight from the MoE equation: each token's output is the gate-weighted   */
 /* sum of its K chosen experts applied to it (no grouping step). logits/idx/gate are outputs;  */
-/* counts (length E) is ADDED TO. Returns the number of tokens with a NaN key.                 */
+/* counts (length E) is ADDED TO; out_acc (optional) receives the double sums before rounding. */
+/* Returns the number of tokens with a NaN key.                                                */
 /* ------------------------------------------------------------------------------------------ */
 
 int64_t oracle_forward(const uint16_t* x, const uint16_t* wr, const float* bias,
                        const uint16_t* w13, const uint16_t* w2, int64_t T, int64_t d, int64_t N,
                        int64_t Z, int64_t K, int64_t I, uint16_t* out, float* logits, int32_t* idx,
-                       float* gate, int32_t* counts) {
+                       float* gate, int32_t* counts, double* out_acc) {
     const int64_t E = N + Z;
     oracle_router_logits(x, wr, T, d, E, logits);
     int64_t bad = oracle_route(logits, bias, T, E, K, idx, gate, counts, NULL);
@@ -341,7 +361,10 @@ int64_t oracle_forward(const uint16_t* x, const uint16_t* wr, const float* bias,
                 for (int64_t c = 0; c < d; ++c) acc[c] += g * bf16_to_double(x[t * d + c]);
             }
         }
-        for (int64_t c = 0; c < d; ++c) out[t * d + c] = oracle_double_to_bf16(acc[c]);
+        for (int64_t c = 0; c < d; ++c) {
+            out[t * d + c] = oracle_double_to_bf16(acc[c]);
+            if (out_acc) out_acc[t * d + c] = acc[c];
+        }
         free(acc); free(yrow);
     }
     return bad;

@@ -68,6 +68,10 @@ MUTATIONS = [
      "double g = (double)gate[t * K + r];\n                double v = (idx[t * K + r] < N)",
      "double g = (double)gate[t * K + 0];\n                double v = (idx[t * K + r] < N)",
      pins.test_combine_weights_rows_and_identity_terms),
+    ("down projection weight transposed",
+     "for (int64_t j = 0; j < I; ++j) acc += hd[j] * bf16_to_double(wd[i * I + j]);",
+     "for (int64_t j = 0; j < I; ++j) acc += hd[j] * bf16_to_double(wd[(j * d + i) % (d * I)]);",
+     pins.test_expert_down_matches_textbook_and_the_full_expert),
     ("softmax denominator off by one term",
      "float S = oracle_sum_spec(e, E);",
      "float S = oracle_sum_spec(e, E - 1);",

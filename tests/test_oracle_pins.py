@@ -271,6 +271,22 @@ def test_expert_rows_match_textbook_swiglu():
         np.testing.assert_allclose(f64(y[r]), yr[0], rtol=2 ** -7, atol=2 ** -8 * np.abs(yr).max())
 
 
+def test_expert_down_matches_textbook_and_the_full_expert():
+    rng = np.random.default_rng(19)
+    M, d, N, I = 30, 48, 3, 64
+    h = bf16(rng.standard_normal((M, I)))
+    w2 = bf16(rng.standard_normal((N, d, I)) * 0.2)
+    re = rng.integers(0, N, M).astype(np.int32)
+    y = oracle.expert_down(h, re, w2)
+    for r in range(M):
+        ref = torch.from_numpy(f64(h[r]) @ f64(w2[re[r]]).T).to(torch.bfloat16).to(torch.float64).numpy()
+        np.testing.assert_allclose(f64(y[r]), ref, rtol=2 ** -7, atol=1e-6)
+    # the down projection of the full expert's own H reproduces its Y bit for bit
+    x, _, w13, w2b = rand_layer(rng, M, d, N, 1, I, w_std=0.3)
+    H, Y = oracle.expert_rows(x, re, w13, w2b)
+    np.testing.assert_array_equal(oracle.expert_down(H, re, w2b), Y)
+
+
 # ------------------------------------------------------------------------------- whole layer
 
 def test_all_zero_expert_picks_return_the_input_exactly():
