@@ -296,11 +296,12 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random-init weights of the LongCat-Flash MoE-layer shape)",
-        "config": {"workload": f"{w.name}: LongCat-Flash-shape MoE layer, prefill batch per GPU",
+        "config": {"workload": f"{w.name}: MoE layer with zero-computation experts, T={T} tokens per GPU",
                    "T": T, "d": d_, "N": w.N, "Z": w.Z, "K": K, "K_e": w.K_e, "I": I_,
                    "router": w.router, "mu": w.mu, "parallelism": f"dp{world}",
                    "step": "forward + counts all-reduce (N>1) + expert-bias update",
-                   "l2": "inputs larger than L2 (38.6 GB expert weights, 201 MB x per step)"},
+                   "l2": f"inputs larger than L2 ({w.weight_bytes() / 1e9:.1f} GB expert weights, "
+                         f"{T * d_ * 2 / 1e6:.0f} MB x per step)"},
         "roofline": roofline,
         "layer_roofline": {"t_roof_ms": round(t_roof * 1e3, 4), "frac": round(t_roof * 1e3 / ms_per_step, 4),
                            "alg_flop": flops, "alg_bytes": bytes_, "ffn_rows_M": M,
@@ -439,7 +440,8 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="prefill", choices=["prefill", "decode", "small", "tiny"])
+    ap.add_argument("--workload", default="prefill",
+                    choices=["prefill", "decode", "small", "tiny", "prefill_ncu", "route_ncu"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time")
     ap.add_argument("--ref-tokens", type=int, default=4, help="tokens per reference-arm step")

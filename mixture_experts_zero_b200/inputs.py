@@ -53,6 +53,14 @@ WORKLOADS = {
     # LongCat-Flash shape, prefill with Zipf(1.1) expert popularity
     "prefill": Workload("prefill", T=16384, d=6144, N=512, Z=256, K=12, K_e=8, I=2048, seed=3,
                         router="zipf"),
+    # the prefill recipe with 32 FFN + 16 zero experts and 4096 tokens (~3.5 GB on the device):
+    # same d, I, K and kernel tiles, small enough for profiler captures
+    "prefill_ncu": Workload("prefill_ncu", T=4096, d=6144, N=32, Z=16, K=12, K_e=8, I=2048, seed=3,
+                            router="zipf"),
+    # LongCat-Flash router shape (E = 768) with 64-wide experts (~4 GB on the device): profiler
+    # captures of the router GEMM, the top-K and the grouping at full routing width
+    "route_ncu": Workload("route_ncu", T=8192, d=6144, N=512, Z=256, K=12, K_e=8, I=64, seed=3,
+                          router="zipf"),
     # bias-control loop: 200 fresh batches of 8192 tokens, routing only
     "bias_loop": Workload("bias_loop", T=8192, d=6144, N=512, Z=256, K=12, K_e=8, I=2048,
                           seed=4, steps=200),

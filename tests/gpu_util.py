@@ -9,10 +9,15 @@ import torch
 import oracle
 from mixture_experts_zero_b200 import inputs
 
-# Output tolerance: max |gpu - oracle| <= 2e-2 * RMS(oracle), with the oracle's output taken
-# before its final rounding to bf16 (two independently rounded bf16 values can differ by one
-# full bf16 step, which at outliers of a heavy-tailed output exceeds 2e-2 * RMS).
+# Output tolerance: |gpu - oracle| <= 2e-2 * RMS(oracle) + half a bf16 step of the oracle value,
+# elementwise, with the oracle's output taken before its final rounding to bf16. The half step
+# is the representation error of the bf16 output itself: beyond ~10 x RMS it alone exceeds
+# 2e-2 * RMS, so a correctly rounded output could not meet the bound without it.
 REL_RMS_TOL = 2e-2
+# Intermediates H and Y: one bf16 step, plus an absolute allowance for fp32 accumulation error
+# where a dot product nearly cancels (relative error is large there although the absolute error
+# is ~1e-6 of the RMS).
+ACC_ABS_TOL = 2.0 ** -14
 
 
 def np_bits(t: torch.Tensor) -> np.ndarray:
@@ -29,12 +34,15 @@ def bf16_ulp(v: np.ndarray) -> np.ndarray:
     return 2.0 ** (np.floor(np.log2(a)) - 7)
 
 
-def assert_within_ulp(got_bits: np.ndarray, ref_bits: np.ndarray, n_ulp: float = 1.0, what=""):
-    """Elementwise |gpu - oracle| <= n_ulp bf16 steps: both round a value computed from the same
-    inputs (fp32 on the GPU, double in the oracle), so they differ by at most one rounding step.
-    Returns the fraction of bit-identical elements."""
+def assert_within_ulp(got_bits: np.ndarray, ref_bits: np.ndarray, n_ulp: float = 1.0, what="",
+                      abs_tol: float = ACC_ABS_TOL):
+    """Elementwise |gpu - oracle| <= n_ulp bf16 steps + abs_tol * RMS(oracle): both round a value
+    computed from the same inputs (fp32 on the GPU, double in the oracle), so they differ by one
+    rounding step plus the fp32 accumulation error. Returns the fraction of bit-identical
+    elements."""
     got, ref = f64(got_bits), f64(ref_bits)
-    lim = n_ulp * bf16_ulp(np.maximum(np.abs(got), np.abs(ref)))
+    rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
+    lim = n_ulp * bf16_ulp(np.maximum(np.abs(got), np.abs(ref))) + abs_tol * rms
     bad = np.abs(got - ref) > lim
     if bad.any():
         i = np.argwhere(bad)[0]
@@ -44,11 +52,17 @@ def assert_within_ulp(got_bits: np.ndarray, ref_bits: np.ndarray, n_ulp: float =
 
 
 def assert_out_close(got_bits: np.ndarray, exact: np.ndarray, tol: float = REL_RMS_TOL, what=""):
-    """Output check against the oracle's double-precision value: max abs error <= tol * RMS."""
+    """Output check against the oracle's double-precision value: elementwise
+    |gpu - exact| <= tol * RMS(exact) + half a bf16 step at |exact|. Returns (max error beyond the
+    half step, RMS)."""
     got = f64(got_bits)
-    rms = float(np.sqrt(np.mean(exact ** 2))) if exact.size else 0.0
-    err = float(np.max(np.abs(got - exact))) if exact.size else 0.0
-    assert err <= tol * rms + 1e-30, f"{what}: max abs err {err:.3e} > {tol} * rms {rms:.3e}"
+    if not exact.size:
+        return 0.0, 0.0
+    rms = float(np.sqrt(np.mean(exact ** 2)))
+    beyond = np.abs(got - exact) - 0.5 * bf16_ulp(exact)
+    err = float(np.max(beyond))
+    assert err <= tol * rms + 1e-30, (
+        f"{what}: max abs err beyond the bf16 half step {err:.3e} > {tol} * rms {rms:.3e}")
     return err, rms
 
 
