@@ -201,6 +201,26 @@ int lc_moe_expert_ffn(const lc_moe_shape* s, const void* x_perm, const int32_t* 
 int lc_moe_combine(const lc_moe_shape* s, const void* x, const void* y, const float* gate,
                    const int32_t* pair_row, void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* lc_moe_permute_noalloc -- lc_moe_permute for callers that cannot allocate device memory: for
+ * example code running inside an engine whose memory planner hands out all device memory up
+ * front and refuses later requests, or a caller with no workspace of its own to pass. The paper
+ * has no counterpart: this entry point is an interface choice of this library. Same arguments and results
+ * as lc_moe_permute, without the workspace: the two grouping tables live in an array inside the
+ * library, reserved on every GPU that loads it until the process exits.
+ *   - Capacity: ceil(T/256) * N <= 131072 (e.g. T <= 65536 with N = 512); larger shapes return
+ *     LC_MOE_ERR_UNSUPPORTED_SHAPE before any launch.
+ *   - status: optional device uint32 (NULL: not reported) that receives the LC_MOE_DEV_* bits,
+ *     OR-ed in; the caller clears it.
+ *   - The first call on a device looks up the array's device address; make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array: calls that overlap on the GPU (different streams without
+ *     ordering, several host threads) race and give wrong groupings. Calls ordered on one stream
+ *     are safe; no state is carried from one call to the next.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+int lc_moe_permute_noalloc(const lc_moe_shape* s, const int32_t* idx, const void* x,
+                           int32_t* offsets, int32_t* row_token, int32_t* pair_row, void* x_perm,
+                           uint32_t* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

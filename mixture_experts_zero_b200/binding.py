@@ -29,7 +29,7 @@ EXPORTED = (
     "lc_moe_abi_version", "lc_moe_strerror", "lc_moe_workspace_bytes", "lc_moe_set_wait_limit_ns",
     "lc_moe_forward", "lc_moe_forward_timed", "lc_moe_route", "lc_moe_bias_update",
     "lc_moe_read_status", "lc_moe_router_logits", "lc_moe_topk", "lc_moe_expert_hist",
-    "lc_moe_permute", "lc_moe_expert_ffn", "lc_moe_combine",
+    "lc_moe_permute", "lc_moe_expert_ffn", "lc_moe_combine", "lc_moe_permute_noalloc",
 )
 
 
@@ -83,6 +83,7 @@ def _configure(L: ctypes.CDLL) -> ctypes.CDLL:
     L.lc_moe_permute.argtypes = [SP, P, P, P, P, P, P, P, SZ, P]
     L.lc_moe_expert_ffn.argtypes = [SP, P, P, P, P, P, P, P, SZ, P]
     L.lc_moe_combine.argtypes = [SP, P, P, P, P, P, P, SZ, P]
+    L.lc_moe_permute_noalloc.argtypes = [SP, P, P, P, P, P, P, P, P]
     return L
 
 
@@ -349,3 +350,27 @@ def lc_moe_combine(x, y, gate, pair_row, out=None, ws=None, stream=None):
     _check(_lib().lc_moe_combine(ctypes.byref(s), _ptr(x), _ptr(y), _ptr(gate), _ptr(pair_row),
                                  _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "lc_moe_combine")
     return out
+
+
+def lc_moe_permute_noalloc(idx, N: int, E: int, x=None, d: int = 64, want_rows: bool = True,
+                           status=None, stream=None):
+    """lc_moe_permute without a workspace (the library's own fixed-size tables; see the header).
+    Returns (offsets[N+1], row_token[T*K], pair_row[T,K], x_perm or None). ``status`` is an
+    optional int32 CUDA tensor of one element that receives device status bits."""
+    T, K = idx.shape
+    _need(idx, torch.int32, (T, K), "idx")
+    dev = idx.device
+    if x is not None:
+        d = x.shape[1]
+        _need(x, torch.bfloat16, (T, d), "x")
+    if status is not None:
+        _need(status, torch.int32, (1,), "status")
+    offsets = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    row_token = torch.empty(T * K, dtype=torch.int32, device=dev)
+    pair_row = torch.empty(T, K, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(T * K, d, dtype=torch.bfloat16, device=dev) if (x is not None and want_rows) else None
+    s = Shape(T, d, N, E - N, K, 64)
+    _check(_lib().lc_moe_permute_noalloc(ctypes.byref(s), _ptr(idx), _ptr(x), _ptr(offsets),
+                                         _ptr(row_token), _ptr(pair_row), _ptr(x_perm), _ptr(status),
+                                         _stream(stream)), "lc_moe_permute_noalloc")
+    return offsets, row_token, pair_row, x_perm

@@ -357,4 +357,20 @@ int lc_moe_combine(const lc_moe_shape* s, const void* x, const void* y, const fl
     return LC_MOE_OK;
 }
 
+int lc_moe_permute_noalloc(const lc_moe_shape* s, const int32_t* idx, const void* x,
+                           int32_t* offsets, int32_t* row_token, int32_t* pair_row, void* x_perm,
+                           uint32_t* status, void* stream) {
+    LC_TRY(check_shape(s));
+    if (!idx || !offsets || !row_token || !pair_row || (x_perm && !x)) return LC_MOE_ERR_INVALID_ARG;
+    if (!permute_noalloc_fits(s->T, s->N)) return LC_MOE_ERR_UNSUPPORTED_SHAPE;
+    for (const void* p : {static_cast<const void*>(idx), x, static_cast<const void*>(x_perm)})
+        if (p && !aligned16(p)) return LC_MOE_ERR_MISALIGNED;
+    LC_TRY(device_ok());
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    LC_CUDA(launch_permute_noalloc(idx, s->T, s->K, s->N, s->N + s->Z, offsets, row_token, pair_row,
+                                   status, st));
+    if (x_perm) LC_CUDA(launch_gather(x, s->T, s->d, s->K, pair_row, x_perm, st));
+    return LC_MOE_OK;
+}
+
 }  // extern "C"

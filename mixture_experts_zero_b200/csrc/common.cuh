@@ -232,6 +232,11 @@ cudaError_t launch_permute(const int32_t* idx, int T, int K, int N, int E, int32
                            uint32_t* status, cudaStream_t st);
 cudaError_t launch_gather(const void* x, int T, int d, int K, const int32_t* pair_row,
                           void* x_perm, cudaStream_t st);
+// Grouping with its tables in a file-scope device array (no caller workspace).
+bool permute_noalloc_fits(int T, int N);
+cudaError_t launch_permute_noalloc(const int32_t* idx, int T, int K, int N, int E, int32_t* offsets,
+                                   int32_t* row_token, int32_t* pair_row, uint32_t* status,
+                                   cudaStream_t st);
 
 cudaError_t launch_combine(const void* x, const void* y, const float* gate,
                            const int32_t* pair_row, int T, int d, int K, void* out,

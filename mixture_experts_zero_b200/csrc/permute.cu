@@ -15,6 +15,8 @@
 //             so rows of an expert are in ascending token order. Writes pair_row and row_token.
 //   gather  : one warp per token copies x_t (16-byte vectors) to each of its FFN rows; x_t is
 //             read once however many FFN experts the token picked.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace lcmoe {
@@ -228,6 +230,60 @@ cudaError_t launch_gather(const void* x, int T, int d, int K, const int32_t* pai
     gather_kernel<<<blocks, GATHER_THREADS, 0, st>>>(static_cast<const uint4*>(x), T, d / 8, K, pair_row,
                                                       static_cast<uint4*>(x_perm));
     return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------------------------
+// Allocation-free grouping: the same three kernels, with the two grouping tables in a file-scope
+// device array instead of a caller-provided workspace, for callers that cannot allocate device
+// memory. Capacity: ceil(T/256) * N <= kNoAllocTableEntries (for example T <= 65536 tokens with
+// N = 512 experts, or T <= 16384 with N = 2048). Every call on a device shares this one array, so
+// calls that overlap on the GPU race on it; calls ordered on one stream do not. Both tables are
+// fully rewritten by every call (counts by the count kernel, bases by the scan kernel), so nothing
+// left over from an earlier call is read.
+// ---------------------------------------------------------------------------------------------
+
+namespace {
+
+constexpr int64_t kNoAllocTableEntries = 131072;  // per table: 512 KB of int32
+__device__ __align__(256) int32_t g_noalloc_tables[2 * kNoAllocTableEntries];
+
+// Device address of g_noalloc_tables on the current device, looked up once per device. In host
+// code the symbol is only a stand-in for the device array; kernels must get this address.
+cudaError_t noalloc_tables_ptr(int32_t** out) {
+    static int32_t* ptrs[64];
+    static cudaError_t errs[64];
+    static std::once_flag flags[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::call_once(flags[dev], [dev] {
+        void* p = nullptr;
+        errs[dev] = cudaGetSymbolAddress(&p, g_noalloc_tables);
+        ptrs[dev] = static_cast<int32_t*>(p);
+    });
+    if (errs[dev] != cudaSuccess) return errs[dev];
+    *out = ptrs[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+bool permute_noalloc_fits(int T, int N) {
+    const int64_t nblk = (static_cast<int64_t>(T) + PB - 1) / PB;
+    return nblk * N <= kNoAllocTableEntries;
+}
+
+cudaError_t launch_permute_noalloc(const int32_t* idx, int T, int K, int N, int E, int32_t* offsets,
+                                   int32_t* row_token, int32_t* pair_row, uint32_t* status,
+                                   cudaStream_t st) {
+    if (!permute_noalloc_fits(T, N)) return cudaErrorInvalidValue;
+    int32_t* tables = nullptr;
+    cudaError_t e = noalloc_tables_ptr(&tables);
+    if (e != cudaSuccess) return e;
+    // launch_permute lays out the count table first and the base table after it, each
+    // ceil(T/256) * N entries: both fit in the array by the capacity check above.
+    return launch_permute(idx, T, K, N, E, offsets, row_token, pair_row, tables, status, st);
 }
 
 }  // namespace lcmoe
