@@ -111,6 +111,7 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": float(np.nanmedian(sm[loaded])) if loaded.any() else float(np.nanmedian(sm)),
                 "sm_max_mhz": float(np.nanmax([num(r[3]) for r in rows])),
+                "power_w": float(np.nanmedian(power[loaded])) if loaded.any() else None,
                 "reasons": sorted(reasons), "samples": int(len(rows)),
                 "samples_under_load": int(loaded.sum())}
 
