@@ -1,0 +1,523 @@
+// umma_pair.cu -- the grouped expert GEMMs on CTA pairs (tcgen05.mma.cta_group::2).
+//
+//   grouped GEMM 1: H[rows_e, I] (bf16) = silu(X_e Wg[e]^T) * (X_e Wu[e]^T)   (SwiGLU epilogue)
+//   grouped GEMM 2: Y[rows_e, d] (bf16) = H_e Wd[e]^T
+// for the N FFN experts of the MoE equation (LongCat-Flash llm-wiki entity page, section 2.1);
+// rows routed to zero-computation experts never reach these GEMMs.
+//
+// A cluster of two CTAs (one per SM) computes 256-row MMA tiles: each CTA holds 128 rows of the
+// A operand and half of the B operand in its own shared memory, and the pair leader issues
+// 256 x N x 16 MMAs that read both; each CTA's TMEM receives its 128 rows of the accumulator.
+// Per SM this halves the B bytes loaded per FLOP compared with a 128-row tile, which lowers the
+// L2-to-SM traffic of the main loop by a third.
+//
+// Roles (256 threads per CTA):
+//   warp 0, one lane, both CTAs  TMA producer: loads this CTA's share of each stage; the bytes
+//                                 complete on the leader's full barrier, where the leader alone
+//                                 posts the expected byte count of the pair;
+//   warp 1, one lane, leader     MMA issuer; tcgen05.commit with a 2-CTA multicast releases the
+//                                 stage in both CTAs and publishes finished accumulators to both;
+//   warp 1, both CTAs            TMEM allocation / deallocation (512 columns, cta_group::2);
+//   warps 4..7, both CTAs        epilogue of this CTA's 128 accumulator lanes; each warp arrives
+//                                 on the leader's accumulator-empty barrier (8 arrivals).
+//
+// Tile kinds, chosen per expert from its row count c_e (as in the single-CTA kernel):
+//   row tiles (c_e >= cold_rows): 256 rows of the expert. GEMM 1: the leader loads 128 gate rows
+//     and its peer the matching 128 up rows of B, so accumulator columns [0, 128) hold gate and
+//     [128, 256) hold up values for every row. GEMM 2: 256 output features, 128 per CTA.
+//   weight tiles (0 < c_e < cold_rows): 256 weight rows (128 per CTA) on the M side and the
+//     expert's rows, rounded up to 64 and split between the CTAs, on the N side. GEMM 1 issues a
+//     gate MMA into columns [0, N) and an up MMA into [128, 128 + N) (N <= 128).
+// The tile list (built on the device from offsets, identically by every CTA) is every row tile
+// in expert order, then every weight tile; tile t goes to cluster t mod (gridDim / 2).
+// Every wait is bounded (lc_moe_set_wait_limit_ns); a wait that runs out raises a CTA-wide abort,
+// records LC_MOE_DEV_WAIT_TIMEOUT, drains in-flight copies and MMAs, and frees TMEM.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace lcmoe {
+
+namespace {
+
+constexpr int HALF_M = 128;                 // A rows per CTA
+constexpr int BK = 64;                      // 64 bf16 = 128 bytes = one swizzle row
+constexpr int STAGES = 4;
+constexpr int A_BYTES = HALF_M * BK * 2;    // 16 KB
+constexpr int B_SLOT = 2 * A_BYTES;         // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_SLOT;
+constexpr int TMEM_COLS = 512;
+constexpr int NUM_THREADS = 256;
+constexpr int TOK_BOX = 32;                 // token rows per TMA box of a weight tile (per CTA)
+constexpr int TOK_ROUND = 2 * TOK_BOX;      // weight-tile N is a multiple of this
+
+enum Mode : int { MODE_SWIGLU = 1, MODE_DOWN = 2 };
+
+struct PairArgs {
+    const int32_t* offsets;  // [n_groups + 1] row offsets
+    __nv_bfloat16* out;      // [rows_cap, ldo]
+    uint32_t* status;
+    uint64_t wait_ns;
+    int64_t rows_cap;
+    int64_t ldo;
+    int n_groups;
+    int kdim;                // reduction length (multiple of 64)
+    int n_out;               // output columns (I or d)
+    int ntiles;              // row tiles per 256-row block of an expert
+    int tile_cols;           // output columns per row tile
+    int b_group_rows;        // rows of the weight matrix per expert
+    int up_off;              // GEMM 1: row offset of Wu inside an expert (= I)
+    int s_tiles;             // weight tiles per cold expert
+    int cold_rows;           // experts with 0 < rows < cold_rows use weight tiles
+};
+
+struct Layout {
+    static constexpr int bars_off = STAGES * STAGE_BYTES;
+    static constexpr int n_bars = 2 * STAGES + 5;  // full, empty, tfull[2], tempty[2], drain
+    static constexpr int misc_off = bars_off + n_bars * 8;
+    static constexpr int table_off = (misc_off + 16 + 15) & ~15;
+    static size_t bytes(int n_groups) { return 1024 + table_off + 3 * static_cast<size_t>(n_groups + 1) * 4; }
+};
+
+struct Tile {
+    int swap;
+    int grp;
+    int64_t row0;
+    int rows;
+    int n0;
+    int ntok;  // weight tile: MMA N
+};
+
+__device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+__device__ __forceinline__ int upper_group(const int32_t* pre, int n, int v) {
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pre[mid] <= v) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    umma_pair_kernel(const __grid_constant__ CUtensorMap mapRows, const __grid_constant__ CUtensorMap mapW,
+                     const __grid_constant__ CUtensorMap mapTok, const PairArgs g) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + Layout::bars_off);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Layout::misc_off);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Layout::misc_off + 4);
+    int32_t* offs_s = reinterpret_cast<int32_t*>(smem + Layout::table_off);
+    int32_t* rpre_s = offs_s + (g.n_groups + 1);
+    int32_t* spre_s = rpre_s + (g.n_groups + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int cluster = blockIdx.x >> 1;
+    const int n_clusters = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 8);  // 4 epilogue warps in each CTA of the pair
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&mapRows);
+        tma_prefetch_desc(&mapW);
+        tma_prefetch_desc(&mapTok);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    for (int e = threadIdx.x; e <= g.n_groups; e += NUM_THREADS) offs_s[e] = g.offsets[e];
+    __syncthreads();
+    if (warp == 2) {
+        int run_r = 0, run_s = 0;
+        if (lane == 0) {
+            rpre_s[0] = 0;
+            spre_s[0] = 0;
+        }
+        for (int base = 0; base < g.n_groups; base += 32) {
+            const int e = base + lane;
+            int nr = 0, ns = 0;
+            if (e < g.n_groups) {
+                int cnt = offs_s[e + 1] - offs_s[e];
+                if (cnt < 0) {
+                    cnt = 0;
+                    set_status(g.status, LC_MOE_DEV_IDX_RANGE);
+                }
+                if (cnt > 0 && cnt < g.cold_rows) ns = g.s_tiles;
+                else nr = (cnt + 2 * HALF_M - 1) / (2 * HALF_M) * g.ntiles;
+            }
+            int ir = nr, is = ns;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int vr = __shfl_up_sync(0xffffffffu, ir, o);
+                const int vs = __shfl_up_sync(0xffffffffu, is, o);
+                if (lane >= o) {
+                    ir += vr;
+                    is += vs;
+                }
+            }
+            if (e < g.n_groups) {
+                rpre_s[e + 1] = run_r + ir;
+                spre_s[e + 1] = run_s + is;
+            }
+            run_r += __shfl_sync(0xffffffffu, ir, 31);
+            run_s += __shfl_sync(0xffffffffu, is, 31);
+        }
+    }
+    __syncthreads();
+    cluster_sync_all();  // both CTAs' barriers are initialised before any cross-CTA signal
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int total_r = rpre_s[g.n_groups];
+    const int total_s = spre_s[g.n_groups];
+    const int total = total_r + total_s;
+    const int nk = g.kdim / BK;
+
+    auto decode = [&](int tile) {
+        Tile tl;
+        tl.swap = tile >= total_r;
+        if (!tl.swap) {
+            const int e = upper_group(rpre_s, g.n_groups, tile);
+            const int local = tile - rpre_s[e];
+            const int mt = local / g.ntiles;
+            tl.grp = e;
+            tl.row0 = static_cast<int64_t>(offs_s[e]) + static_cast<int64_t>(mt) * 2 * HALF_M;
+            tl.rows = min(2 * HALF_M, offs_s[e + 1] - offs_s[e] - mt * 2 * HALF_M);
+            tl.n0 = (local - mt * g.ntiles) * g.tile_cols;
+            tl.ntok = 0;
+        } else {
+            const int idx = tile - total_r;
+            const int e = upper_group(spre_s, g.n_groups, idx);
+            tl.grp = e;
+            tl.row0 = offs_s[e];
+            tl.rows = offs_s[e + 1] - offs_s[e];
+            tl.n0 = (idx - spre_s[e]) * 2 * HALF_M;
+            tl.ntok = (tl.rows + TOK_ROUND - 1) / TOK_ROUND * TOK_ROUND;
+        }
+        return tl;
+    };
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------------- TMA producer (both CTAs) --
+        const uint64_t pol_stream = l2_policy_evict_first();
+        const uint64_t pol_normal = l2_policy_evict_normal();
+        int s = 0;
+        uint32_t ph = 0;
+        int issued = 0;
+        bool ok = true;
+        for (int tile = cluster; tile < total && ok; tile += n_clusters) {
+            const Tile tl = decode(tile);
+            const int tok_rows = tl.ntok / 2;  // this CTA's share of the N side
+            uint32_t cta_bytes;
+            if (!tl.swap) cta_bytes = A_BYTES + A_BYTES;
+            else cta_bytes = (MODE == MODE_SWIGLU ? 2 : 1) * A_BYTES + tok_rows * BK * 2;
+            const int wbase = tl.grp * g.b_group_rows;
+            for (int kb = 0; kb < nk; ++kb) {
+                if (!mbar_wait(&empty[s], ph ^ 1u, g.wait_ns, abort_flag, g.status)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* sa = smem + s * STAGE_BYTES;
+                uint8_t* sb = sa + A_BYTES;
+                const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+                if (leader) mbar_arrive_expect_tx(&full[s], 2 * cta_bytes);
+                const int kx = kb * BK;
+                if (!tl.swap) {
+                    tma_load_2d_pair(sa, &mapRows, bar, kx, static_cast<int32_t>(tl.row0 + rank * HALF_M), pol_normal);
+                    // GEMM 1: leader gate rows, peer up rows; GEMM 2: 128 output features each
+                    const int wrow = (MODE == MODE_SWIGLU) ? wbase + tl.n0 + static_cast<int>(rank) * g.up_off
+                                                           : wbase + tl.n0 + static_cast<int>(rank) * HALF_M;
+                    tma_load_2d_pair(sb, &mapW, bar, kx, wrow, pol_normal);
+                } else {
+                    const int wrow = wbase + tl.n0 + static_cast<int>(rank) * HALF_M;
+                    tma_load_2d_pair(sa, &mapW, bar, kx, wrow, pol_stream);
+                    uint8_t* st = sb;
+                    if (MODE == MODE_SWIGLU) {
+                        tma_load_2d_pair(sb, &mapW, bar, kx, wrow + g.up_off, pol_stream);
+                        st = sb + A_BYTES;
+                    }
+                    const int64_t t0 = tl.row0 + static_cast<int64_t>(rank) * tok_rows;
+                    for (int b = 0; b < tok_rows; b += TOK_BOX)
+                        tma_load_2d_pair(st + b * 128, &mapTok, bar, kx, static_cast<int32_t>(t0 + b), pol_normal);
+                }
+                ++issued;
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+        if (!ok && leader) {
+            for (int i = 0; i < STAGES && i < issued; ++i) {
+                if (s == 0) {
+                    s = STAGES - 1;
+                    ph ^= 1u;
+                } else {
+                    --s;
+                }
+                wait_drain(&full[s], ph, g.wait_ns);
+            }
+        }
+    } else if (warp == 1 && lane == 0 && leader) {
+        // ------------------------------------------------------- MMA issuer (leader only) --
+        int s = 0;
+        uint32_t ph = 0;
+        int acc = 0;
+        uint32_t aph = 0;
+        bool ok = true;
+        for (int tile = cluster; tile < total && ok; tile += n_clusters) {
+            const Tile tl = decode(tile);
+            const uint32_t idesc = idesc_bf16_f32(2 * HALF_M, tl.swap ? tl.ntok : 2 * HALF_M);
+            if (!mbar_wait(&tempty[acc], aph ^ 1u, g.wait_ns, abort_flag, g.status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
+            for (int kb = 0; kb < nk; ++kb) {
+                if (!mbar_wait(&full[s], ph, g.wait_ns, abort_flag, g.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint8_t* sa = smem + s * STAGE_BYTES;
+                const uint64_t ad = sw128_kmajor_desc(smem_u32(sa));
+                const uint64_t bd = sw128_kmajor_desc(smem_u32(sa + A_BYTES));
+                if (MODE == MODE_SWIGLU && tl.swap) {
+                    const uint64_t td = sw128_kmajor_desc(smem_u32(sa + 2 * A_BYTES));
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        umma_bf16_pair(d_tmem, ad + 2 * kk, td + 2 * kk, idesc, (kb | kk) != 0);
+                        umma_bf16_pair(d_tmem + 128, bd + 2 * kk, td + 2 * kk, idesc, (kb | kk) != 0);
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        umma_bf16_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                }
+                umma_commit_pair(&empty[s], 0x3);
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            if (!ok) break;
+            umma_commit_pair(&tfull[acc], 0x3);
+            acc ^= 1;
+            if (acc == 0) aph ^= 1u;
+        }
+        umma_commit_pair(drain, 0x1);
+        wait_drain(drain, 0, g.wait_ns);
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue (both CTAs) --
+        const int q = warp - 4;
+        int acc = 0;
+        uint32_t aph = 0;
+        __nv_bfloat16* out = g.out;
+        for (int tile = cluster; tile < total; tile += n_clusters) {
+            const Tile tl = decode(tile);
+            if (!mbar_wait(&tfull[acc], aph, g.wait_ns, abort_flag, g.status)) break;
+            tc_fence_after();
+            const uint32_t tb =
+                tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * 256);
+            const int i = q * 32 + lane;  // TMEM lane of this thread
+            if (!tl.swap) {
+                const int r = static_cast<int>(rank) * HALF_M + i;  // row within the 256-row tile
+                const int64_t grow = tl.row0 + r;
+                const bool valid = r < tl.rows && grow < g.rows_cap;
+                if (MODE == MODE_SWIGLU) {
+                    for (int c = 0; c < HALF_M; c += 32) {
+                        uint32_t gv[32], uv[32];
+                        tmem_ld_32x32b_x32(tb + c, gv);
+                        tmem_ld_32x32b_x32(tb + HALF_M + c, uv);
+                        tmem_ld_wait();
+                        const int f0 = tl.n0 + c;
+                        if (valid && f0 < g.n_out) {
+                            uint32_t pk[16];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                pk[j] = pack_bf16x2(silu_mul(__uint_as_float(gv[2 * j]), __uint_as_float(uv[2 * j])),
+                                                    silu_mul(__uint_as_float(gv[2 * j + 1]), __uint_as_float(uv[2 * j + 1])));
+                            uint4* d4 = reinterpret_cast<uint4*>(out + grow * g.ldo + f0);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                d4[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                        }
+                    }
+                } else {
+                    for (int c = 0; c < 2 * HALF_M; c += 32) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(tb + c, v);
+                        tmem_ld_wait();
+                        const int f0 = tl.n0 + c;
+                        if (valid && f0 < g.n_out) {
+                            uint32_t pk[16];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
+                            uint4* d4 = reinterpret_cast<uint4*>(out + grow * g.ldo + f0);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                d4[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                        }
+                    }
+                }
+            } else {
+                // weight tile: lane = output feature, column = row of the expert's group
+                const int feat = tl.n0 + static_cast<int>(rank) * HALF_M + i;
+                const bool fvalid = feat < g.n_out;
+                for (int c0 = 0; c0 < tl.ntok; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tb + c0, v);
+                    if (MODE == MODE_SWIGLU) {
+                        uint32_t uv[32];
+                        tmem_ld_32x32b_x32(tb + HALF_M + c0, uv);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int row = c0 + j;
+                            const int64_t grow = tl.row0 + row;
+                            if (fvalid && row < tl.rows && grow < g.rows_cap)
+                                out[grow * g.ldo + feat] = __float2bfloat16_rn(
+                                    silu_mul(__uint_as_float(v[j]), __uint_as_float(uv[j])));
+                        }
+                    } else {
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int row = c0 + j;
+                            const int64_t grow = tl.row0 + row;
+                            if (fvalid && row < tl.rows && grow < g.rows_cap)
+                                out[grow * g.ldo + feat] = __float2bfloat16_rn(__uint_as_float(v[j]));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+            acc ^= 1;
+            if (acc == 0) aph ^= 1u;
+        }
+    }
+
+    __syncthreads();
+    cluster_sync_all();  // the leader's MMAs have finished reading the peer's shared memory
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
+template <int MODE>
+cudaError_t launch_pair(const CUtensorMap& mr, const CUtensorMap& mw, const CUtensorMap& mt,
+                        const PairArgs& args, int grid, cudaStream_t st) {
+    const size_t smem = Layout::bytes(args.n_groups);
+    static int configured[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && configured[dev] < static_cast<int>(smem)) {
+        int max_optin = 0;
+        e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return e;
+        if (static_cast<int>(smem) > max_optin) return cudaErrorInvalidValue;
+        e = cudaFuncSetAttribute(umma_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_optin);
+        if (e != cudaSuccess) return e;
+        configured[dev] = max_optin;
+    }
+    umma_pair_kernel<MODE><<<grid, NUM_THREADS, smem, st>>>(mr, mw, mt, args);
+    return cudaGetLastError();
+}
+
+int pair_grid(const DevInfo* di) { return (di->sm_count / 2) * 2; }
+
+}  // namespace
+
+cudaError_t launch_grouped_swiglu(const void* x_perm, int64_t rows_cap, const int32_t* offsets,
+                                  int N, const void* w13, int d, int I, void* h, uint32_t* status,
+                                  cudaStream_t st) {
+    const DevInfo* di = current_device_info();
+    if (!di) return cudaErrorUnknown;
+    CUtensorMap mr, mw, mt;
+    if (!make_tma_map_2d(&mr, x_perm, static_cast<uint64_t>(rows_cap), d, HALF_M)) return cudaErrorInvalidValue;
+    if (!make_tma_map_2d(&mw, w13, static_cast<uint64_t>(N) * 2 * I, d, HALF_M)) return cudaErrorInvalidValue;
+    if (!make_tma_map_2d(&mt, x_perm, static_cast<uint64_t>(rows_cap), d, TOK_BOX)) return cudaErrorInvalidValue;
+    PairArgs a{};
+    a.offsets = offsets;
+    a.out = static_cast<__nv_bfloat16*>(h);
+    a.status = status;
+    a.wait_ns = wait_limit_ns();
+    a.rows_cap = rows_cap;
+    a.ldo = I;
+    a.n_groups = N;
+    a.kdim = d;
+    a.n_out = I;
+    a.ntiles = (I + HALF_M - 1) / HALF_M;  // 128 features (gate + up) per row tile
+    a.tile_cols = HALF_M;
+    a.b_group_rows = 2 * I;
+    a.up_off = I;
+    a.s_tiles = (I + 2 * HALF_M - 1) / (2 * HALF_M);  // 256 features per weight tile
+    a.cold_rows = 128;  // weight-tile N <= 128 keeps gate and up in one 256-column accumulator
+    return launch_pair<MODE_SWIGLU>(mr, mw, mt, a, pair_grid(di), st);
+}
+
+cudaError_t launch_grouped_down(const void* h, int64_t rows_cap, const int32_t* offsets, int N,
+                                const void* w2, int d, int I, void* y, uint32_t* status,
+                                cudaStream_t st) {
+    const DevInfo* di = current_device_info();
+    if (!di) return cudaErrorUnknown;
+    CUtensorMap mr, mw, mt;
+    if (!make_tma_map_2d(&mr, h, static_cast<uint64_t>(rows_cap), I, HALF_M)) return cudaErrorInvalidValue;
+    if (!make_tma_map_2d(&mw, w2, static_cast<uint64_t>(N) * d, I, HALF_M)) return cudaErrorInvalidValue;
+    if (!make_tma_map_2d(&mt, h, static_cast<uint64_t>(rows_cap), I, TOK_BOX)) return cudaErrorInvalidValue;
+    PairArgs a{};
+    a.offsets = offsets;
+    a.out = static_cast<__nv_bfloat16*>(y);
+    a.status = status;
+    a.wait_ns = wait_limit_ns();
+    a.rows_cap = rows_cap;
+    a.ldo = d;
+    a.n_groups = N;
+    a.kdim = I;
+    a.n_out = d;
+    a.ntiles = (d + 2 * HALF_M - 1) / (2 * HALF_M);  // 256 output features per row tile
+    a.tile_cols = 2 * HALF_M;
+    a.b_group_rows = d;
+    a.up_off = 0;
+    a.s_tiles = (d + 2 * HALF_M - 1) / (2 * HALF_M);
+    a.cold_rows = 256;
+    return launch_pair<MODE_DOWN>(mr, mw, mt, a, pair_grid(di), st);
+}
+
+}  // namespace lcmoe
