@@ -21,15 +21,20 @@
 //   warps 4..7, both CTAs        epilogue of this CTA's 128 accumulator lanes; each warp arrives
 //                                 on the leader's accumulator-empty barrier (8 arrivals).
 //
-// Tile kinds, chosen per expert from its row count c_e (as in the single-CTA kernel):
-//   row tiles (c_e >= cold_rows): 256 rows of the expert. GEMM 1: the leader loads 128 gate rows
-//     and its peer the matching 128 up rows of B, so accumulator columns [0, 128) hold gate and
-//     [128, 256) hold up values for every row. GEMM 2: 256 output features, 128 per CTA.
-//   weight tiles (0 < c_e < cold_rows): 256 weight rows (128 per CTA) on the M side and the
-//     expert's rows, rounded up to 64 and split between the CTAs, on the N side. GEMM 1 issues a
-//     gate MMA into columns [0, N) and an up MMA into [128, 128 + N) (N <= 128).
-// The tile list (built on the device from offsets, identically by every CTA) is every row tile
-// in expert order, then every weight tile; tile t goes to cluster t mod (gridDim / 2).
+// Tile kinds:
+//   row tiles: 256 rows of one expert. GEMM 1: the leader loads 128 gate rows and its peer the
+//     matching 128 up rows of B, so accumulator columns [0, 128) hold gate and [128, 256) hold up
+//     values for every row. GEMM 2: 256 output features, 128 per CTA.
+//   weight tiles ("swap"): 256 weight rows (128 per CTA) on the M side and up to 256 rows of one
+//     expert, rounded up to 64 and split between the CTAs, on the N side. GEMM 1 issues a gate MMA
+//     into columns [0, N) and an up MMA into [128, 128 + N) (N <= 128).
+// Per expert with c_e rows: below cold_rows it is "cold" and runs as weight tiles only; otherwise
+// it runs floor(c_e / 256) row tiles, and its leftover rows run as one more row tile if there are
+// at least rem_rows of them, else as weight tiles (N rounded up to 64): an expert's padding rows
+// stay below 128 for GEMM 1 (rem_rows = 128) and below 64 for GEMM 2 (rem_rows = 256). The tile list (built on the device from offsets, identically
+// by every CTA) is: for each hot expert in order, its row tiles then its leftover weight tiles
+// (whose weights were just read by its row tiles and are still in L2); then the weight tiles of
+// every cold expert. Tile t goes to cluster t mod (gridDim / 2).
 // Every wait is bounded (lc_moe_set_wait_limit_ns); a wait that runs out raises a CTA-wide abort,
 // records LC_MOE_DEV_WAIT_TIMEOUT, drains in-flight copies and MMAs, and frees TMEM.
 #include <cudaTypedefs.h>
@@ -69,15 +74,24 @@ struct PairArgs {
     int tile_cols;           // output columns per row tile
     int b_group_rows;        // rows of the weight matrix per expert
     int up_off;              // GEMM 1: row offset of Wu inside an expert (= I)
-    int s_tiles;             // weight tiles per cold expert
-    int cold_rows;           // experts with 0 < rows < cold_rows use weight tiles
+    int s_tiles;             // weight tiles per group of rows (256 output features each)
+    int cold_rows;           // experts with 0 < rows < cold_rows use weight tiles only
+    int rem_rows;            // an expert's rows past its last full 256-row tile: fewer than this
+                             // run as weight tiles, otherwise as one more row tile
 };
+
+// Epilogue transpose tile of one warp: 32 rows x 32 features (bf16), 64 bytes per row, its four
+// 16-byte chunks stored at chunk ^ ((row >> 1) & 3), so that both the writes (one row at a time)
+// and the reads (8 rows per 128-byte phase) hit distinct banks.
+constexpr int XPOSE_ROW = 64;
+constexpr int XPOSE_WARP = 32 * XPOSE_ROW;
 
 struct Layout {
     static constexpr int bars_off = STAGES * STAGE_BYTES;
     static constexpr int n_bars = 2 * STAGES + 5;  // full, empty, tfull[2], tempty[2], drain
     static constexpr int misc_off = bars_off + n_bars * 8;
-    static constexpr int table_off = (misc_off + 16 + 15) & ~15;
+    static constexpr int xpose_off = (misc_off + 16 + 127) & ~127;
+    static constexpr int table_off = xpose_off + 4 * XPOSE_WARP;
     static size_t bytes(int n_groups) { return 1024 + table_off + 3 * static_cast<size_t>(n_groups + 1) * 4; }
 };
 
@@ -158,39 +172,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     for (int e = threadIdx.x; e <= g.n_groups; e += NUM_THREADS) offs_s[e] = g.offsets[e];
     __syncthreads();
     if (warp == 2) {
-        int run_r = 0, run_s = 0;
+        // per expert: tiles of the hot part (row tiles + weight tiles of the leftover rows) and
+        // weight tiles of a cold expert; exclusive prefix sums of both
+        int run_h = 0, run_c = 0;
         if (lane == 0) {
             rpre_s[0] = 0;
             spre_s[0] = 0;
         }
         for (int base = 0; base < g.n_groups; base += 32) {
             const int e = base + lane;
-            int nr = 0, ns = 0;
+            int nh = 0, nc = 0;
             if (e < g.n_groups) {
                 int cnt = offs_s[e + 1] - offs_s[e];
                 if (cnt < 0) {
                     cnt = 0;
                     set_status(g.status, LC_MOE_DEV_IDX_RANGE);
                 }
-                if (cnt > 0 && cnt < g.cold_rows) ns = g.s_tiles;
-                else nr = (cnt + 2 * HALF_M - 1) / (2 * HALF_M) * g.ntiles;
+                if (cnt > 0 && cnt < g.cold_rows) {
+                    nc = g.s_tiles;
+                } else if (cnt > 0) {
+                    const int nfull = cnt / (2 * HALF_M);
+                    const int rem = cnt - nfull * 2 * HALF_M;
+                    const bool rem_row = rem >= g.rem_rows;
+                    nh = (nfull + (rem_row ? 1 : 0)) * g.ntiles + ((rem > 0 && !rem_row) ? g.s_tiles : 0);
+                }
             }
-            int ir = nr, is = ns;
+            int ih = nh, ic = nc;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int vr = __shfl_up_sync(0xffffffffu, ir, o);
-                const int vs = __shfl_up_sync(0xffffffffu, is, o);
+                const int vh = __shfl_up_sync(0xffffffffu, ih, o);
+                const int vc = __shfl_up_sync(0xffffffffu, ic, o);
                 if (lane >= o) {
-                    ir += vr;
-                    is += vs;
+                    ih += vh;
+                    ic += vc;
                 }
             }
             if (e < g.n_groups) {
-                rpre_s[e + 1] = run_r + ir;
-                spre_s[e + 1] = run_s + is;
+                rpre_s[e + 1] = run_h + ih;
+                spre_s[e + 1] = run_c + ic;
             }
-            run_r += __shfl_sync(0xffffffffu, ir, 31);
-            run_s += __shfl_sync(0xffffffffu, is, 31);
+            run_h += __shfl_sync(0xffffffffu, ih, 31);
+            run_c += __shfl_sync(0xffffffffu, ic, 31);
         }
     }
     __syncthreads();
@@ -205,19 +227,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 
     auto decode = [&](int tile) {
         Tile tl;
-        tl.swap = tile >= total_r;
-        if (!tl.swap) {
+        if (tile < total_r) {
+            // hot expert: its row tiles, then weight tiles for the rows past its last row tile
             const int e = upper_group(rpre_s, g.n_groups, tile);
             const int local = tile - rpre_s[e];
-            const int mt = local / g.ntiles;
+            const int cnt = offs_s[e + 1] - offs_s[e];
+            const int nfull = cnt / (2 * HALF_M);
+            const int rem = cnt - nfull * 2 * HALF_M;
+            const int nrow = (nfull + (rem >= g.rem_rows ? 1 : 0)) * g.ntiles;
             tl.grp = e;
-            tl.row0 = static_cast<int64_t>(offs_s[e]) + static_cast<int64_t>(mt) * 2 * HALF_M;
-            tl.rows = min(2 * HALF_M, offs_s[e + 1] - offs_s[e] - mt * 2 * HALF_M);
-            tl.n0 = (local - mt * g.ntiles) * g.tile_cols;
-            tl.ntok = 0;
+            if (local < nrow) {
+                const int mt = local / g.ntiles;
+                tl.swap = 0;
+                tl.row0 = static_cast<int64_t>(offs_s[e]) + static_cast<int64_t>(mt) * 2 * HALF_M;
+                tl.rows = min(2 * HALF_M, cnt - mt * 2 * HALF_M);
+                tl.n0 = (local - mt * g.ntiles) * g.tile_cols;
+                tl.ntok = 0;
+            } else {
+                tl.swap = 1;
+                tl.row0 = static_cast<int64_t>(offs_s[e]) + static_cast<int64_t>(nfull) * 2 * HALF_M;
+                tl.rows = rem;
+                tl.n0 = (local - nrow) * 2 * HALF_M;
+                tl.ntok = (rem + TOK_ROUND - 1) / TOK_ROUND * TOK_ROUND;
+            }
         } else {
+            // cold expert: weight tiles only
             const int idx = tile - total_r;
             const int e = upper_group(spre_s, g.n_groups, idx);
+            tl.swap = 1;
             tl.grp = e;
             tl.row0 = offs_s[e];
             tl.rows = offs_s[e + 1] - offs_s[e];
@@ -393,9 +430,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     }
                 }
             } else {
-                // weight tile: lane = output feature, column = row of the expert's group
-                const int feat = tl.n0 + static_cast<int>(rank) * HALF_M + i;
-                const bool fvalid = feat < g.n_out;
+                // weight tile: lane = output feature, column = row of the expert's group. Each
+                // 32 x 32 block goes through shared memory transposed, so that every thread then
+                // stores 32 consecutive features of one row as four 16-byte vectors.
+                uint8_t* xp = smem + Layout::xpose_off + q * XPOSE_WARP;
+                const int f0 = tl.n0 + static_cast<int>(rank) * HALF_M + q * 32;  // warp's first feature
                 for (int c0 = 0; c0 < tl.ntok; c0 += 32) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(tb + c0, v);
@@ -404,23 +443,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         tmem_ld_32x32b_x32(tb + HALF_M + c0, uv);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int row = c0 + j;
-                            const int64_t grow = tl.row0 + row;
-                            if (fvalid && row < tl.rows && grow < g.rows_cap)
-                                out[grow * g.ldo + feat] = __float2bfloat16_rn(
-                                    silu_mul(__uint_as_float(v[j]), __uint_as_float(uv[j])));
-                        }
+                        for (int j = 0; j < 32; ++j)
+                            v[j] = __float_as_uint(silu_mul(__uint_as_float(v[j]), __uint_as_float(uv[j])));
                     } else {
                         tmem_ld_wait();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int row = c0 + j;
-                            const int64_t grow = tl.row0 + row;
-                            if (fvalid && row < tl.rows && grow < g.rows_cap)
-                                out[grow * g.ldo + feat] = __float2bfloat16_rn(__uint_as_float(v[j]));
-                        }
                     }
+                    // lane = feature f0 + lane, v[j] = value for row c0 + j
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        *reinterpret_cast<__nv_bfloat16*>(
+                            xp + j * XPOSE_ROW + ((((lane >> 3) ^ (j >> 1)) & 3) << 4) + (lane & 7) * 2) =
+                            __float2bfloat16_rn(__uint_as_float(v[j]));
+                    __syncwarp();
+                    const int row = c0 + lane;
+                    const int64_t grow = tl.row0 + row;
+                    if (row < tl.rows && grow < g.rows_cap && f0 < g.n_out) {
+                        uint4* dst = reinterpret_cast<uint4*>(out + grow * g.ldo + f0);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            dst[k] = *reinterpret_cast<const uint4*>(
+                                xp + lane * XPOSE_ROW + (((k ^ (lane >> 1)) & 3) << 4));
+                    }
+                    __syncwarp();
                 }
             }
             tc_fence_before();
@@ -488,7 +532,9 @@ cudaError_t launch_grouped_swiglu(const void* x_perm, int64_t rows_cap, const in
     a.b_group_rows = 2 * I;
     a.up_off = I;
     a.s_tiles = (I + 2 * HALF_M - 1) / (2 * HALF_M);  // 256 features per weight tile
-    a.cold_rows = 128;  // weight-tile N <= 128 keeps gate and up in one 256-column accumulator
+    // weight-tile N <= 128 keeps gate and up in one 256-column accumulator
+    a.cold_rows = 128;
+    a.rem_rows = 128;
     return launch_pair<MODE_SWIGLU>(mr, mw, mt, a, pair_grid(di), st);
 }
 
@@ -517,6 +563,7 @@ cudaError_t launch_grouped_down(const void* h, int64_t rows_cap, const int32_t* 
     a.up_off = 0;
     a.s_tiles = (d + 2 * HALF_M - 1) / (2 * HALF_M);
     a.cold_rows = 256;
+    a.rem_rows = 256;
     return launch_pair<MODE_DOWN>(mr, mw, mt, a, pair_grid(di), st);
 }
 
