@@ -14,6 +14,23 @@ namespace {
 
 constexpr int COMBINE_THREADS = 256;
 
+// Loads in flight per lane: two 16-byte column chunks (c and c + 32) of PB picks at a time.
+constexpr int PB = 4;
+
+__device__ __forceinline__ void fma_row(float (&acc)[8], float g, const uint4& v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        acc[2 * j] = __fmaf_rn(g, bf16lo(w[j]), acc[2 * j]);
+        acc[2 * j + 1] = __fmaf_rn(g, bf16hi(w[j]), acc[2 * j + 1]);
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
+    return make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                      pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+}
+
 __global__ void __launch_bounds__(COMBINE_THREADS)
     combine_kernel(const uint4* __restrict__ x, const uint4* __restrict__ y,
                    const float* __restrict__ gate, const int32_t* __restrict__ pair_row, int T,
@@ -29,30 +46,44 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
         }
         const bool any_zero = __any_sync(0xffffffffu, lane < K && my_row < 0);
         const uint4* xt = x + static_cast<int64_t>(t) * d8;
-        for (int c0 = 0; c0 < d8; c0 += 32) {  // warp-uniform trip count
-            const int c = c0 + lane;
-            const bool in = c < d8;
-            uint4 xv = make_uint4(0, 0, 0, 0);
-            if (in && any_zero) xv = __ldg(xt + c);
-            float acc[8];
+        for (int c0 = 0; c0 < d8; c0 += 64) {  // warp-uniform trip count
+            const int ca = c0 + lane, cb = c0 + 32 + lane;
+            const bool ina = ca < d8, inb = cb < d8;
+            uint4 xa = make_uint4(0, 0, 0, 0), xb = xa;
+            if (any_zero) {
+                if (ina) xa = __ldg(xt + ca);
+                if (inb) xb = __ldg(xt + cb);
+            }
+            float acc_a[8], acc_b[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-            for (int r = 0; r < K; ++r) {
-                const float g = __shfl_sync(0xffffffffu, my_g, r);
-                const int row = __shfl_sync(0xffffffffu, my_row, r);
-                if (!in) continue;
-                const uint4 v = (row >= 0) ? __ldg(y + static_cast<int64_t>(row) * d8 + c) : xv;
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            for (int j = 0; j < 8; ++j) acc_a[j] = acc_b[j] = 0.0f;
+            for (int r0 = 0; r0 < K; r0 += PB) {
+                float g[PB];
+                int row[PB];
+                uint4 va[PB], vb[PB];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    acc[2 * j] = __fmaf_rn(g, bf16lo(w[j]), acc[2 * j]);
-                    acc[2 * j + 1] = __fmaf_rn(g, bf16hi(w[j]), acc[2 * j + 1]);
+                for (int u = 0; u < PB; ++u) {
+                    g[u] = __shfl_sync(0xffffffffu, my_g, (r0 + u) & 31);
+                    row[u] = __shfl_sync(0xffffffffu, my_row, (r0 + u) & 31);
+                }
+#pragma unroll
+                for (int u = 0; u < PB; ++u) {
+                    const bool pick = r0 + u < K;
+                    const uint4* yr = y + static_cast<int64_t>(row[u] < 0 ? 0 : row[u]) * d8;
+                    va[u] = (pick && row[u] >= 0 && ina) ? __ldg(yr + ca) : xa;
+                    vb[u] = (pick && row[u] >= 0 && inb) ? __ldg(yr + cb) : xb;
+                }
+                // rank order: pick r0, r0 + 1, ... each one fused multiply-add per element
+#pragma unroll
+                for (int u = 0; u < PB; ++u) {
+                    if (r0 + u < K) {
+                        fma_row(acc_a, g[u], va[u]);
+                        fma_row(acc_b, g[u], vb[u]);
+                    }
                 }
             }
-            if (in)
-                out[static_cast<int64_t>(t) * d8 + c] =
-                    make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                               pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+            if (ina) out[static_cast<int64_t>(t) * d8 + ca] = pack8(acc_a);
+            if (inb) out[static_cast<int64_t>(t) * d8 + cb] = pack8(acc_b);
         }
     }
 }

@@ -164,17 +164,24 @@ __global__ void __launch_bounds__(GATHER_THREADS)
         const uint32_t dests = __ballot_sync(0xffffffffu, my_row >= 0);
         if (!dests) continue;
         const uint4* src = x + static_cast<int64_t>(t) * d8;
-        for (int c0 = 0; c0 < d8; c0 += 32) {  // warp-uniform trip count
-            const int c = c0 + lane;
-            const bool in = c < d8;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (in) v = __ldg(src + c);
+        for (int c0 = 0; c0 < d8; c0 += 128) {  // warp-uniform trip count; 4 loads in flight
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int c = c0 + 32 * u + lane;
+                v[u] = c < d8 ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+            }
             uint32_t m = dests;
             while (m) {
                 const int r = __ffs(m) - 1;
                 m &= m - 1;
                 const int row = __shfl_sync(0xffffffffu, my_row, r);
-                if (in) x_perm[static_cast<int64_t>(row) * d8 + c] = v;
+                uint4* dst = x_perm + static_cast<int64_t>(row) * d8;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + 32 * u + lane;
+                    if (c < d8) dst[c] = v[u];
+                }
             }
         }
     }

@@ -2,7 +2,9 @@
 // controller (LongCat-Flash llm-wiki entity page, section 2.1; softmax gate: section 2.3.2).
 //
 //   topk      : per token, s = softmax(z) over all E = N + Z experts; key_i = s_i + b_i;
-//               the K largest keys in descending order (equal keys: lower index first);
+//               the K largest keys in descending order (equal keys: lower index first), found by
+//               K rounds of a warp-wide max over each lane's best untaken key, then a warp-wide
+//               min over the indices of the lanes holding that key;
 //               gate_r = s_sel[r] / (s_sel[0] + ... + s_sel[K-1]); optional histogram of picks.
 //   hist      : T_i, the number of picks of each expert (the T_i of the bias-update equation).
 //   bias      : b_i += mu * (K_e/(K N) - T_i/(K T_all)) for all E experts.
@@ -22,16 +24,16 @@ namespace lcmoe {
 
 namespace {
 
-// fp32 constants of the exp above, from ln 2 and 1/k!
+// fp32 constants of the exp above, from ln 2 and 1/k!. Branch-free: the argument is clamped to
+// [-86, 88] for the arithmetic and the result is replaced by 0 below -86, +inf above 88 and the
+// argument itself when it is NaN (the same values as the specification's early returns).
 __device__ __forceinline__ float exp_spec(float u) {
     const float LOG2E = 0x1.715476p+0f;     // 1/ln 2, rounded to fp32
     const float LN2_HI = 0x1.62e4p-1f;      // ln 2 rounded to 16 fraction bits (exact)
     const float LN2_LO = 0x1.7f7d1cp-20f;   // ln 2 - LN2_HI, rounded to fp32
-    if (u != u) return u;
-    if (u < -86.0f) return 0.0f;
-    if (u > 88.0f) return __int_as_float(0x7f800000);
-    const float n = rintf(__fmul_rn(u, LOG2E));
-    float r = __fmaf_rn(-n, LN2_HI, u);
+    const float uc = fminf(fmaxf(u, -86.0f), 88.0f);
+    const float n = rintf(__fmul_rn(uc, LOG2E));
+    float r = __fmaf_rn(-n, LN2_HI, uc);
     r = __fmaf_rn(-n, LN2_LO, r);
     float p = 0x1.a01a02p-13f;              // 1/7!
     p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);   // 1/6!
@@ -42,14 +44,10 @@ __device__ __forceinline__ float exp_spec(float u) {
     p = __fmaf_rn(p, r, 1.0f);              // 1/1!
     p = __fmaf_rn(p, r, 1.0f);              // 1/0!
     const float scale = __int_as_float((static_cast<int>(n) + 127) << 23);  // 2^n, normal
-    return __fmul_rn(p, scale);
-}
-
-// (key, index) order of the selection: larger key first, equal keys lower index first.
-__device__ __forceinline__ bool better(float ka, int ia, float kb, int ib) {
-    if (ib < 0) return ia >= 0;
-    if (ia < 0) return false;
-    return ka > kb || (ka == kb && ia < ib);
+    float e = __fmul_rn(p, scale);
+    e = (u < -86.0f) ? 0.0f : e;
+    e = (u > 88.0f) ? __int_as_float(0x7f800000) : e;
+    return (u != u) ? u : e;
 }
 
 constexpr int TOPK_THREADS = 256;  // 8 warps, one token per warp at a time
@@ -59,20 +57,17 @@ __global__ void __launch_bounds__(TOPK_THREADS)
     topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E,
                 int K, int32_t* __restrict__ idx, float* __restrict__ gate,
                 int32_t* __restrict__ counts, uint32_t* __restrict__ status) {
-    extern __shared__ int32_t s_hist[];
+    extern __shared__ int32_t smem_i[];
+    int32_t* s_hist = smem_i;                                   // [E]
+    float* s_bias = reinterpret_cast<float*>(smem_i + E);      // [E]
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const bool do_hist = counts != nullptr;
-    if (do_hist)
-        for (int i = threadIdx.x; i < E; i += TOPK_THREADS) s_hist[i] = 0;
-    __syncthreads();
-
-    float b[VPL];
-#pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-        const int i = lane + 32 * j;
-        b[j] = (i < E) ? bias[i] : 0.0f;
+    for (int i = threadIdx.x; i < E; i += TOPK_THREADS) {
+        s_hist[i] = 0;
+        s_bias[i] = bias[i];
     }
+    __syncthreads();
 
     const int warps_total = gridDim.x * (TOPK_THREADS / 32);
     for (int t = blockIdx.x * (TOPK_THREADS / 32) + warp; t < T; t += warps_total) {
@@ -103,16 +98,20 @@ __global__ void __launch_bounds__(TOPK_THREADS)
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) part = __fadd_rn(part, __shfl_xor_sync(0xffffffffu, part, o));
         const float S = part;
-        // scores s_i and keys s_i + b_i
-        float key[VPL];
+        // scores s_i = e_i / S and keys s_i + b_i, the keys as order-preserving unsigned integers
+        // (no key is -0: scores are >= +0, and +0 + -0 rounds to +0; 0 is below every key)
+        uint32_t ku[VPL];
         bool nan_key = false;
 #pragma unroll
         for (int j = 0; j < VPL; ++j) {
             const int i = lane + 32 * j;
+            ku[j] = 0;
             if (i < E) {
                 v[j] = __fdiv_rn(v[j], S);
-                key[j] = __fadd_rn(v[j], b[j]);
-                nan_key |= (key[j] != key[j]);
+                const float key = __fadd_rn(v[j], s_bias[i]);
+                nan_key |= (key != key);
+                const uint32_t kb = __float_as_uint(key);
+                ku[j] = (kb & 0x80000000u) ? ~kb : (kb | 0x80000000u);
             }
         }
         if (__any_sync(0xffffffffu, nan_key)) {
@@ -124,46 +123,44 @@ __global__ void __launch_bounds__(TOPK_THREADS)
             }
             continue;
         }
-        // K rounds of warp arg-max over (key, index)
+        // K rounds of warp arg-max over (key, index); each lane keeps its best two untaken
+        // (key, index, score) and rescans only when both are taken.
         uint64_t taken = 0;
-        float lk = 0.0f, ls = 0.0f;
-        int li = -1;
-        auto local_best = [&]() {
-            li = -1;
+        uint32_t k1 = 0, k2 = 0;
+        int i1 = 0x7fffffff, i2 = 0x7fffffff;
+        float s1 = 0.0f, s2 = 0.0f;
+        auto top2 = [&]() {
+            k1 = k2 = 0;
+            i1 = i2 = 0x7fffffff;
 #pragma unroll
             for (int j = 0; j < VPL; ++j) {
                 const int i = lane + 32 * j;
-                if (i < E && !((taken >> j) & 1ull) && (li < 0 || key[j] > lk)) {
-                    lk = key[j];
-                    ls = v[j];
-                    li = i;
+                if (!((taken >> j) & 1ull)) {  // ku = 0 (past E) never wins
+                    if (ku[j] > k1) {
+                        k2 = k1; i2 = i1; s2 = s1;
+                        k1 = ku[j]; i1 = i; s1 = v[j];
+                    } else if (ku[j] > k2) {
+                        k2 = ku[j]; i2 = i; s2 = v[j];
+                    }
                 }
             }
         };
-        local_best();
+        top2();
         int my_idx = 0;
         float my_s = 0.0f;
         for (int r = 0; r < K; ++r) {
-            float bk = lk, bs = ls;
-            int bi = li;
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) {
-                const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-                const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (better(ok, oi, bk, bi)) {
-                    bk = ok;
-                    bs = os;
-                    bi = oi;
-                }
-            }
+            const uint32_t m = __reduce_max_sync(0xffffffffu, k1);
+            const int w = __reduce_min_sync(0xffffffffu, k1 == m ? static_cast<uint32_t>(i1) : 0x7fffffffu);
+            const float ws = __shfl_sync(0xffffffffu, s1, w & 31);
             if (lane == r) {
-                my_idx = bi;
-                my_s = bs;
+                my_idx = w;
+                my_s = ws;
             }
-            if (bi >= 0 && (bi & 31) == lane) {
-                taken |= 1ull << (bi >> 5);
-                local_best();
+            if ((w & 31) == lane) {
+                taken |= 1ull << (w >> 5);
+                k1 = k2; i1 = i2; s1 = s2;
+                k2 = 0; i2 = 0x7fffffff;
+                if (k1 == 0) top2();
             }
         }
         // renormalise over the K chosen, summing in rank order
@@ -193,7 +190,7 @@ cudaError_t launch_topk_t(const float* logits, const float* bias, int T, int E, 
     const int cap = sm_count * 4;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    const size_t smem = counts ? static_cast<size_t>(E) * sizeof(int32_t) : 0;
+    const size_t smem = 2 * static_cast<size_t>(E) * sizeof(int32_t);
     topk_kernel<VPL><<<blocks, TOPK_THREADS, smem, st>>>(logits, bias, T, E, K, idx, gate, counts,
                                                           status);
     return cudaGetLastError();
