@@ -222,23 +222,50 @@ def run_ours(args):
     M = int(c[: w.N].sum())
     touched = int((c[: w.N] > 0).sum())
 
-    # ---- end to end through the public API: pinned host x -> device, layer, out -> pinned host
+    # ---- end to end through the public API: every step copies its x from pinned host memory to
+    # the device and its output back to pinned host memory. The copies run on a copy stream and
+    # overlap the compute of the neighbouring steps (H2D of step i+1 and D2H of step i-1 during
+    # step i), with double-buffered device x and out.
     x_host = x.cpu().pin_memory()
-    out_host = torch.empty(T, w.d, dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(x)
-    for _ in range(max(1, args.warmup // 2)):
-        x_dev.copy_(x_host, non_blocking=True)
-        step(xin=x_dev)
-        out_host.copy_(out, non_blocking=True)
+    out_host = [torch.empty(T, w.d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(x) for _ in range(2)]
+    out_dev = [torch.empty_like(out) for _ in range(2)]
+    copy = torch.cuda.Stream(dev)
+    h2d_done = [torch.cuda.Event() for _ in range(2)]
+    fwd_done = [torch.cuda.Event() for _ in range(2)]
+    d2h_done = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_steps(n):
+        with torch.cuda.stream(copy):
+            copy.wait_stream(stream)  # earlier work on the buffers has finished
+            x_dev[0].copy_(x_host, non_blocking=True)
+            h2d_done[0].record(copy)
+        for i in range(n):
+            b = i & 1
+            if i + 1 < n:
+                with torch.cuda.stream(copy):
+                    if i >= 1:
+                        copy.wait_event(fwd_done[b ^ 1])  # step i-1 has finished reading x_dev[b^1]
+                    x_dev[b ^ 1].copy_(x_host, non_blocking=True)
+                    h2d_done[b ^ 1].record(copy)
+            stream.wait_event(h2d_done[b])
+            if i >= 2:
+                stream.wait_event(d2h_done[b])  # step i-2's output has left out_dev[b]
+            step(xin=x_dev[b], o=out_dev[b])
+            fwd_done[b].record(stream)
+            with torch.cuda.stream(copy):
+                copy.wait_event(fwd_done[b])
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+                d2h_done[b].record(copy)
+        stream.wait_stream(copy)
+
+    e2e_steps(max(2, args.warmup // 2))
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(1, min(args.steps, 20))
+    e2e_steps_n = max(2, min(args.steps, 40))
     e0.record(stream)
-    for _ in range(e2e_steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        step(xin=x_dev)
-        out_host.copy_(out, non_blocking=True)
+    e2e_steps(e2e_steps_n)
     e1.record(stream)
     barrier()
     e2e_ms = e0.elapsed_time(e1)
@@ -246,7 +273,7 @@ def run_ours(args):
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     e2e_ms = float(t.item())
-    e2e_value = T * world * e2e_steps / (e2e_ms / 1e3)
+    e2e_value = T * world * e2e_steps_n / (e2e_ms / 1e3)
 
     # ---- roofline of each stage (algorithmic work only)
     peaks, peak_src = load_peaks()
@@ -311,8 +338,12 @@ def run_ours(args):
                            "ffn_per_token": round(M / T, 4)},
         "stages": stages,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": int(x.numel() * 2),
-                "d2h_bytes_per_step": int(out.numel() * 2), "steps": e2e_steps},
+                "d2h_bytes_per_step": int(out.numel() * 2), "steps": e2e_steps_n,
+                "copies": "pinned host x -> device and out -> pinned host every step, on a copy "
+                          "stream overlapping the neighbouring steps' compute"},
         "gpu_launches": int(args.steps * (sum(KERNELS_PER_STAGE) + 1)),
+        "gpu_launches_note": "kernels of this library inside the device-timed region: "
+                             f"{sum(KERNELS_PER_STAGE)} per forward + 1 bias update, per step",
         "clocks": ClockSampler.summarize(clock_rows),
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
