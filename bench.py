@@ -7,6 +7,7 @@ LongCat-Flash-shape prefill batch (T=16384 tokens per GPU, d=6144, 512 FFN exper
 256 zero experts, K=12, K_e=8, Zipf(1.1) expert popularity), synthetic data.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --sweep ffn_rows|hist      (kernel sweeps, one JSON line per case)
 
 Prints one JSON line (rank 0). ``--impl reference`` times the CPU oracle (test infrastructure) on a
 bounded sample of the same workload instead.
@@ -335,7 +336,10 @@ def run_ours(args):
                            "alg_flop": flops, "alg_bytes": bytes_, "ffn_rows_M": M,
                            "experts_touched": touched,
                            "zero_expert_share": round(float(c[w.N:].sum()) / (T * K), 4),
-                           "ffn_per_token": round(M / T, 4)},
+                           "ffn_per_token": round(M / T, 4),
+                           "ffn_experts_by_rows": {
+                               f"[{lo},{hi})": int(((c[:w.N] >= lo) & (c[:w.N] < hi)).sum())
+                               for lo, hi in ((1, 128), (128, 256), (256, 512), (512, 1024), (1024, T + 1))}},
         "stages": stages,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": int(x.numel() * 2),
                 "d2h_bytes_per_step": int(out.numel() * 2), "steps": e2e_steps_n,
@@ -466,6 +470,81 @@ def run_reference(args):
     }), flush=True)
 
 
+# ------------------------------------------------------------------------------ kernel sweeps --
+
+FFN_ROWS_CASES = ((16, 512), (32, 512), (64, 512), (96, 512), (128, 512), (160, 512), (192, 512),
+                  (256, 512), (320, 256), (384, 256), (512, 256), (768, 128), (1024, 128),
+                  (2048, 64), (4096, 32))
+
+
+def run_sweep(args):
+    """Kernel sweeps outside the step, one JSON line per case (one GPU, device-timed, L2 flushed
+    with a 256 MB write before every timed call, median of the timed calls).
+
+    ffn_rows: the two grouped expert GEMMs (lc_moe_expert_ffn) at the prefill shape (d=6144,
+        I=2048) with c rows for each of n experts, against max(6*M*d*I FLOP / sustained TC peak,
+        (3*n*d*I + 2*M*(2d+I)) * 2 bytes / HBM).
+    hist: the expert-count histogram over idx[2^24, 12] (805 MB of int32), against HBM."""
+    import torch
+    from mixture_experts_zero_b200 import binding as B
+
+    peaks, peak_src = load_peaks()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(256 * 2 ** 20 // 4, device=dev)
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    g = torch.Generator(device=dev).manual_seed(7)
+    if args.sweep == "hist":
+        T, K, E = 1 << 24, 12, 768
+        idx = torch.randint(0, E, (T, K), generator=g, device=dev, dtype=torch.int32)
+        counts = torch.zeros(E, dtype=torch.int32, device=dev)
+        ms = timed(lambda: B.lc_moe_expert_hist(idx, E, counts=counts), 10)
+        gbs = idx.numel() * 4 / ms / 1e6
+        print(json.dumps({"sweep": "hist", "T": T, "K": K, "n_bins": E, "ms": round(ms, 4),
+                          "achieved_gbs": round(gbs, 1), "peak_gbs": peaks["hbm_gbs"],
+                          "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_source": peak_src}), flush=True)
+        return
+    d, I = 6144, 2048
+    n_max = max(n for _, n in FFN_ROWS_CASES)
+    w13 = torch.empty(n_max, 2 * I, d, dtype=torch.bfloat16, device=dev)
+    w2 = torch.empty(n_max, d, I, dtype=torch.bfloat16, device=dev)
+    for e in range(n_max):
+        w13[e].normal_(0.0, 0.02, generator=g)
+        w2[e].normal_(0.0, 0.02, generator=g)
+    tc, hbm = peaks["bf16_tflops_sustained"] * 1e12, peaks["hbm_gbs"] * 1e9
+    for c, n in FFN_ROWS_CASES:
+        M = c * n
+        x = torch.empty(M, d, dtype=torch.bfloat16, device=dev).normal_(generator=g)
+        offsets = torch.arange(n + 1, dtype=torch.int32, device=dev) * c
+        h = torch.empty(M, I, dtype=torch.bfloat16, device=dev)
+        y = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
+        ms = timed(lambda: B.lc_moe_expert_ffn(x, offsets, w13[:n], w2[:n], M, 1, h=h, y=y), 8)
+        flop = 6 * M * d * I
+        bytes_ = (3 * n * d * I + 2 * M * (2 * d + I)) * 2
+        roof = max(flop / tc, bytes_ / hbm) * 1e3
+        print(json.dumps({"sweep": "ffn_rows", "rows_per_expert": c, "experts": n, "ms": round(ms, 3),
+                          "roof_ms": round(roof, 3), "frac": round(roof / ms, 3),
+                          "tflops": round(flop / ms / 1e9, 1), "gbs": round(bytes_ / ms / 1e6, 1),
+                          "peak_source": peak_src}), flush=True)
+        del x, h, y
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -477,7 +556,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time")
     ap.add_argument("--ref-tokens", type=int, default=4, help="tokens per reference-arm step")
+    ap.add_argument("--sweep", choices=["ffn_rows", "hist"], default=None,
+                    help="run a kernel sweep instead of the step (one GPU)")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":

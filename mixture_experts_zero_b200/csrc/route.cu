@@ -197,6 +197,7 @@ cudaError_t launch_topk_t(const float* logits, const float* bias, int T, int E, 
 }
 
 constexpr int HIST_THREADS = 512;
+constexpr int HIST_UNROLL = 4;
 
 __global__ void __launch_bounds__(HIST_THREADS)
     hist_kernel(const int32_t* __restrict__ idx, int64_t n, int n_bins, int32_t* __restrict__ counts,
@@ -208,13 +209,24 @@ __global__ void __launch_bounds__(HIST_THREADS)
     const int64_t stride = static_cast<int64_t>(gridDim.x) * HIST_THREADS;
     const int64_t n4 = n / 4;
     const int4* idx4 = reinterpret_cast<const int4*>(idx);
-    for (int64_t p = static_cast<int64_t>(blockIdx.x) * HIST_THREADS + threadIdx.x; p < n4; p += stride) {
-        const int4 q = __ldg(idx4 + p);
-        const int vals[4] = {q.x, q.y, q.z, q.w};
+    // HIST_UNROLL 16-byte loads in flight per thread before their shared-memory atomics
+    for (int64_t p0 = static_cast<int64_t>(blockIdx.x) * HIST_THREADS + threadIdx.x; p0 < n4;
+         p0 += HIST_UNROLL * stride) {
+        int4 q[HIST_UNROLL];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            if (vals[j] >= 0 && vals[j] < n_bins) atomicAdd(&s_hist[vals[j]], 1);
-            else bad = true;
+        for (int u = 0; u < HIST_UNROLL; ++u) {
+            const int64_t p = p0 + u * stride;
+            q[u] = p < n4 ? __ldg(idx4 + p) : make_int4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < HIST_UNROLL; ++u) {
+            if (p0 + u * stride >= n4) break;
+            const int vals[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (vals[j] >= 0 && vals[j] < n_bins) atomicAdd(&s_hist[vals[j]], 1);
+                else bad = true;
+            }
         }
     }
     for (int64_t p = n4 * 4 + static_cast<int64_t>(blockIdx.x) * HIST_THREADS + threadIdx.x; p < n; p += stride) {
