@@ -45,6 +45,14 @@ def configure(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_forward.argtypes = [P, P, P, P, P, I64, I64, I64, I64, I64, I64, P, P, P, P, P, P]
     L.oracle_forward.restype = I64
     L.oracle_bias_update.argtypes = [P, P, I64, I64, I64, I64, I64, ctypes.c_float]
+    L.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+    L.oracle_e4m3_to_double.restype = ctypes.c_double
+    L.oracle_float_to_e4m3.argtypes = [ctypes.c_float]
+    L.oracle_float_to_e4m3.restype = ctypes.c_uint8
+    L.oracle_quantize_rows_e4m3.argtypes = [P, I64, I64, P, P]
+    L.oracle_expert_rows_fp8.argtypes = [P, P, P, I64, I64, I64, P, P, P, P, P]
+    L.oracle_forward_fp8.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, P, P, P, P, P, P]
+    L.oracle_forward_fp8.restype = I64
     return L
 
 
@@ -217,3 +225,74 @@ def bias_update(bias: np.ndarray, counts: np.ndarray, T_all: int, N: int, Z: int
     assert b.shape == (N + Z,) and counts.shape == (N + Z,)
     lib().oracle_bias_update(_p(b), _p(counts), T_all, N, Z, K, K_e, ctypes.c_float(mu))
     return b
+
+
+# ------------------------------------------------------------------------------ FP8 experts --
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """E4M3 codes (uint8) -> float64 values (NaN for the NaN codes)."""
+    L = lib()
+    table = np.array([L.oracle_e4m3_to_double(c) for c in range(256)], dtype=np.float64)
+    return table[np.asarray(codes, dtype=np.uint8)]
+
+
+def f32_to_e4m3(v) -> np.ndarray:
+    """float32 -> nearest E4M3 code, ties to even, saturating at 448 (one rounding)."""
+    L = lib()
+    flat = np.asarray(v, dtype=np.float32).ravel()
+    out = np.fromiter((L.oracle_float_to_e4m3(float(a)) for a in flat), dtype=np.uint8,
+                      count=flat.size)
+    return out.reshape(np.shape(v))
+
+
+def quantize_rows_e4m3(src: np.ndarray):
+    """Row-wise E4M3 quantisation of bf16 bits [R, C]: s = amax/448 (fp32), q = E4M3(x / s).
+    Returns (q uint8 [R, C], s float32 [R])."""
+    src = _c(src, np.uint16)
+    R, C = src.shape
+    q = np.empty((R, C), dtype=np.uint8)
+    s = np.empty(R, dtype=np.float32)
+    lib().oracle_quantize_rows_e4m3(_p(src), R, C, _p(q), _p(s))
+    return q, s
+
+
+def expert_rows_fp8(xq: np.ndarray, sx: np.ndarray, row_expert: np.ndarray, w13q: np.ndarray,
+                    w13_scale: np.ndarray, w2: np.ndarray, want_h: bool = True):
+    """FP8 SwiGLU expert of each row: gate/up from E4M3 codes with row scales, down in bf16.
+    w13q is [N, 2I, d] uint8 with w13_scale [N, 2I]; w2 is [N, d, I] bf16 bits."""
+    xq = _c(xq, np.uint8); sx = _c(sx, np.float32); row_expert = _c(row_expert, np.int32)
+    w13q = _c(w13q, np.uint8); w13_scale = _c(w13_scale, np.float32); w2 = _c(w2, np.uint16)
+    M, d = xq.shape
+    n, two_i, d2 = w13q.shape
+    I = two_i // 2
+    assert d2 == d and w2.shape == (n, d, I) and w13_scale.shape == (n, two_i)
+    assert sx.shape == (M,) and row_expert.shape == (M,)
+    if M and (row_expert.min() < 0 or row_expert.max() >= n):
+        raise ValueError("row_expert out of range")
+    h = np.empty((M, I), dtype=np.uint16) if want_h else None
+    y = np.empty((M, d), dtype=np.uint16)
+    lib().oracle_expert_rows_fp8(_p(xq), _p(sx), _p(row_expert), M, d, I, _p(w13q), _p(w13_scale),
+                                 _p(w2), _p(h), _p(y))
+    return h, y
+
+
+def forward_fp8(x, wr, bias, w13q, w13_scale, w2, N: int, Z: int, K: int,
+                counts: np.ndarray | None = None):
+    """The layer with FP8 gate/up projections (token rows quantised per row). Same return
+    value as ``forward``."""
+    x = _c(x, np.uint16); wr = _c(wr, np.uint16); bias = _c(bias, np.float32)
+    w13q = _c(w13q, np.uint8); w13_scale = _c(w13_scale, np.float32); w2 = _c(w2, np.uint16)
+    T, d = x.shape
+    E = N + Z
+    I = w2.shape[2]
+    assert wr.shape == (E, d) and w13q.shape == (N, 2 * I, d) and w2.shape == (N, d, I)
+    assert w13_scale.shape == (N, 2 * I)
+    out = np.empty((T, d), dtype=np.uint16)
+    logits = np.empty((T, E), dtype=np.float32)
+    idx = np.empty((T, K), dtype=np.int32)
+    gate = np.empty((T, K), dtype=np.float32)
+    cnt = np.zeros(E, dtype=np.int32) if counts is None else _c(counts, np.int32)
+    acc = np.empty((T, d), dtype=np.float64)
+    bad = lib().oracle_forward_fp8(_p(x), _p(wr), _p(bias), _p(w13q), _p(w13_scale), _p(w2), T, d,
+                                   N, Z, K, I, _p(out), _p(logits), _p(idx), _p(gate), _p(cnt), _p(acc))
+    return dict(out=out, out_exact=acc, logits=logits, idx=idx, gate=gate, counts=cnt, bad=int(bad))

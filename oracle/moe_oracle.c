@@ -371,6 +371,141 @@ int64_t oracle_forward(const uint16_t* x, const uint16_t* wr, const float* bias,
 }
 
 /* ------------------------------------------------------------------------------------------ */
+/* FP8 experts. The LongCat-Flash llm-wiki entity page, section 5 (inference and deployment),   */
+/* lists FP8/BF16 quantisation among the system-level optimisations and an FP8 deployment on   */
+/* one node in its measured-performance table; it gives no scaling scheme. Reading used here:  */
+/* the gate and up projections run on E4M3 operands, each weight row (output feature) and each */
+/* token row carrying one fp32 scale (amax / 448); the down projection stays bf16.             */
+/*                                                                                              */
+/* E4M3 as the OCP 8-bit floating point format defines it: sign, 4 exponent bits (bias 7),      */
+/* 3 mantissa bits; exponent field 0 holds subnormals m * 2^-9; S.1111.111 is NaN; there is no  */
+/* infinity; the largest finite magnitude is 448 (1.110b * 2^8).                                */
+/* ------------------------------------------------------------------------------------------ */
+
+double oracle_e4m3_to_double(uint8_t c) {
+    const int e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double v = (e == 0) ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return (c & 0x80) ? -v : v;
+}
+
+/* Nearest E4M3 value of v, ties to the even mantissa; finite magnitudes above 448 give 448
+ * (saturation), NaN gives the NaN code. The sign of v is kept, zero included. */
+uint8_t oracle_float_to_e4m3(float v) {
+    if (isnan(v)) return 0x7F;
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs((double)v);
+    if (a >= 448.0) return sign | 0x7E;
+    int code;
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal spacing 2^-9; a count of 8 is the smallest normal, whose code is also 8 */
+        code = (int)nearbyint(a * 512.0);
+    } else {
+        int ex;
+        frexp(a, &ex);            /* a = f * 2^ex, f in [0.5, 1) */
+        int e = ex - 1;           /* a in [2^e, 2^(e+1)), e in -6..8 */
+        double q = nearbyint(ldexp(a, 3 - e));   /* mantissa steps of 2^(e-3): q in [8, 16] */
+        if (q == 16.0) {
+            e += 1;
+            q = 8.0;
+        }
+        code = ((e + 7) << 3) | ((int)q - 8);
+    }
+    return sign | (uint8_t)code;
+}
+
+/* Row-wise quantisation of a bf16 matrix [R, C]: amax = max_k |x_k|; s = amax / 448 as one fp32
+ * division (s = 1 for an all-zero row); q_k = E4M3(x_k / s) with x_k / s one fp32 division.
+ * Then x_k ~ s * q_k. */
+void oracle_quantize_rows_e4m3(const uint16_t* src, int64_t R, int64_t C, uint8_t* dst,
+                               float* scale) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < C; ++k) {
+            const float a = fabsf((float)bf16_to_double(src[r * C + k]));
+            if (a > amax) amax = a;
+        }
+        const float s = (amax > 0.0f) ? amax / 448.0f : 1.0f;
+        scale[r] = s;
+        for (int64_t k = 0; k < C; ++k) {
+            const float q = (float)bf16_to_double(src[r * C + k]) / s;
+            dst[r * C + k] = oracle_float_to_e4m3(q);
+        }
+    }
+}
+
+/* FP8 experts on grouped rows: row r holds the E4M3 codes xq[r, :] of its token with scale
+ * sx[r]; W13q[e] = [Wg; Wu] codes [2I, d] with one scale per row in w13_scale[e * 2I + j].
+ *   G_j = sum_k (sx qx_k) (sg_j qg_jk),  U_j likewise   (double)
+ *   H_j = bf16( G_j sigmoid(G_j) U_j ),  Y = bf16( H Wd[e]^T )  (Wd bf16, as in step 7). */
+void oracle_expert_rows_fp8(const uint8_t* xq, const float* sx, const int32_t* row_expert,
+                            int64_t M, int64_t d, int64_t I, const uint8_t* w13q,
+                            const float* w13_scale, const uint16_t* w2, uint16_t* h, uint16_t* y) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < M; ++r) {
+        const int64_t e = row_expert[r];
+        const uint8_t* wg = w13q + e * 2 * I * d;
+        const uint8_t* wu = wg + I * d;
+        const float* sg = w13_scale + e * 2 * I;
+        const float* su = sg + I;
+        double* xd = (double*)malloc((size_t)d * sizeof(double));
+        double* hd = (double*)malloc((size_t)I * sizeof(double));
+        for (int64_t k = 0; k < d; ++k) xd[k] = (double)sx[r] * oracle_e4m3_to_double(xq[r * d + k]);
+        for (int64_t j = 0; j < I; ++j) {
+            double G = 0.0, U = 0.0;
+            for (int64_t k = 0; k < d; ++k) {
+                G += xd[k] * ((double)sg[j] * oracle_e4m3_to_double(wg[j * d + k]));
+                U += xd[k] * ((double)su[j] * oracle_e4m3_to_double(wu[j * d + k]));
+            }
+            const double silu = G / (1.0 + exp(-G));
+            uint16_t hb = oracle_double_to_bf16(silu * U);
+            if (h) h[r * I + j] = hb;
+            hd[j] = bf16_to_double(hb);
+        }
+        down_row(hd, w2 + e * d * I, d, I, y + r * d);
+        free(xd); free(hd);
+    }
+}
+
+/* The layer with FP8 experts: as oracle_forward, with each token row quantised by
+ * oracle_quantize_rows_e4m3 and every FFN pick computed by oracle_expert_rows_fp8. Routing and
+ * the zero-computation experts use the bf16 x unchanged. */
+int64_t oracle_forward_fp8(const uint16_t* x, const uint16_t* wr, const float* bias,
+                           const uint8_t* w13q, const float* w13_scale, const uint16_t* w2,
+                           int64_t T, int64_t d, int64_t N, int64_t Z, int64_t K, int64_t I,
+                           uint16_t* out, float* logits, int32_t* idx, float* gate,
+                           int32_t* counts, double* out_acc) {
+    const int64_t E = N + Z;
+    oracle_router_logits(x, wr, T, d, E, logits);
+    int64_t bad = oracle_route(logits, bias, T, E, K, idx, gate, counts, NULL);
+    uint8_t* xq = (uint8_t*)malloc((size_t)(T * d));
+    float* sx = (float*)malloc((size_t)T * sizeof(float));
+    oracle_quantize_rows_e4m3(x, T, d, xq, sx);
+    for (int64_t t = 0; t < T; ++t) {
+        double* acc = (double*)calloc((size_t)d, sizeof(double));
+        uint16_t* yrow = (uint16_t*)malloc((size_t)d * sizeof(uint16_t));
+        for (int64_t r = 0; r < K; ++r) {
+            const int32_t e = idx[t * K + r];
+            const double g = (double)gate[t * K + r];
+            if (e < N) {
+                oracle_expert_rows_fp8(xq + t * d, sx + t, &e, 1, d, I, w13q, w13_scale, w2, NULL, yrow);
+                for (int64_t c = 0; c < d; ++c) acc[c] += g * bf16_to_double(yrow[c]);
+            } else {
+                for (int64_t c = 0; c < d; ++c) acc[c] += bf16_to_double(x[t * d + c]) * g;  /* E_i(x) = x */
+            }
+        }
+        for (int64_t c = 0; c < d; ++c) {
+            out[t * d + c] = oracle_double_to_bf16(acc[c]);
+            if (out_acc) out_acc[t * d + c] = acc[c];
+        }
+        free(acc); free(yrow);
+    }
+    free(xq); free(sx);
+    return bad;
+}
+
+/* ------------------------------------------------------------------------------------------ */
 /* Bias update (section 2.1, dynamic computation-budget control):                              */
 /*   b_i <- b_i + mu * (K_e/K * 1/N - T_i/(K * T_all))   for all E = N + Z experts,            */
 /* as these fp32 operations, each rounded once:                                                */

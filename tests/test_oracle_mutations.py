@@ -13,6 +13,7 @@ import pytest
 
 import oracle
 from oracle import build as oracle_build
+import tests.test_oracle_fp8 as fp8pins
 import tests.test_oracle_pins as pins
 
 MUTATIONS = [
@@ -76,6 +77,26 @@ MUTATIONS = [
      "float S = oracle_sum_spec(e, E);",
      "float S = oracle_sum_spec(e, E - 1);",
      pins.test_scores_are_the_softmax_over_all_experts),
+    ("FP8: up projection scaled with the gate row's scale",
+     "U += xd[k] * ((double)su[j] * oracle_e4m3_to_double(wu[j * d + k]));",
+     "U += xd[k] * ((double)sg[j] * oracle_e4m3_to_double(wu[j * d + k]));",
+     fp8pins.test_fp8_experts_reduce_to_the_bf16_oracle_on_exact_inputs),
+    ("FP8: E4M3 exponent bias 8 instead of 7",
+     "ldexp(1.0 + m / 8.0, e - 7);",
+     "ldexp(1.0 + m / 8.0, e - 8);",
+     fp8pins.test_code_table_matches_the_format_definition),
+    ("FP8: ties rounded away from zero",
+     "double q = nearbyint(ldexp(a, 3 - e));",
+     "double q = round(ldexp(a, 3 - e));",
+     fp8pins.test_ties_go_to_the_even_code_and_large_values_saturate),
+    ("FP8: row scale for a largest code of 240",
+     "const float s = (amax > 0.0f) ? amax / 448.0f : 1.0f;",
+     "const float s = (amax > 0.0f) ? amax / 240.0f : 1.0f;",
+     fp8pins.test_row_quantisation_scale_and_error_bound),
+    ("FP8: no saturation at 448",
+     "if (a >= 448.0) return sign | 0x7E;",
+     "if (a >= 480.0) return sign | 0x7F;",
+     fp8pins.test_ties_go_to_the_even_code_and_large_values_saturate),
 ]
 
 
