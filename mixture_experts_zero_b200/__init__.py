@@ -13,7 +13,9 @@ from .binding import (  # noqa: F401,E402
     lc_moe_expert_ffn,
     lc_moe_expert_hist,
     lc_moe_forward,
+    lc_moe_forward_fp8,
     lc_moe_permute,
+    lc_moe_quantize_e4m3,
     lc_moe_read_status,
     lc_moe_route,
     lc_moe_router_logits,

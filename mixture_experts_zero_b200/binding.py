@@ -21,7 +21,7 @@ OK = 0
 ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_WORKSPACE_TOO_SMALL, ERR_NOT_SM100 = 1, 2, 3, 4
 ERR_CUDA, ERR_DEVICE_STATUS, ERR_TIMEOUT, ERR_MISALIGNED = 5, 6, 7, 8
 DEV_IDX_RANGE, DEV_NAN_KEY, DEV_WAIT_TIMEOUT, DEV_DUP_PICK = 0x1, 0x2, 0x4, 0x8
-OP_FORWARD, OP_ROUTE, OP_PERMUTE, OP_STATUS = 0, 1, 2, 3
+OP_FORWARD, OP_ROUTE, OP_PERMUTE, OP_STATUS, OP_FORWARD_FP8 = 0, 1, 2, 3, 4
 NUM_STAGES = 7
 STAGE_NAMES = ("router_gemm", "topk", "permute", "gather", "gemm1_swiglu", "gemm2_down", "combine")
 
@@ -30,6 +30,7 @@ EXPORTED = (
     "lc_moe_forward", "lc_moe_forward_timed", "lc_moe_route", "lc_moe_bias_update",
     "lc_moe_read_status", "lc_moe_router_logits", "lc_moe_topk", "lc_moe_expert_hist",
     "lc_moe_permute", "lc_moe_expert_ffn", "lc_moe_combine", "lc_moe_permute_noalloc",
+    "lc_moe_quantize_e4m3", "lc_moe_forward_fp8", "lc_moe_forward_fp8_timed",
 )
 
 
@@ -84,6 +85,10 @@ def _configure(L: ctypes.CDLL) -> ctypes.CDLL:
     L.lc_moe_expert_ffn.argtypes = [SP, P, P, P, P, P, P, P, SZ, P]
     L.lc_moe_combine.argtypes = [SP, P, P, P, P, P, P, SZ, P]
     L.lc_moe_permute_noalloc.argtypes = [SP, P, P, P, P, P, P, P, P]
+    L.lc_moe_quantize_e4m3.argtypes = [P, I64, I32, P, P, P]
+    fwd8 = [SP, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+    L.lc_moe_forward_fp8.argtypes = fwd8
+    L.lc_moe_forward_fp8_timed.argtypes = fwd8 + [ctypes.POINTER(P)]
     return L
 
 
@@ -179,13 +184,69 @@ def lc_moe_forward(x, wr, bias, w13, w2, K: int, out=None, idx=None, gate=None, 
     if events is None:
         _check(_lib().lc_moe_forward(*args), "lc_moe_forward")
     else:
-        if len(events) != NUM_STAGES + 1:
-            raise ValueError(f"events: need {NUM_STAGES + 1} CUDA events")
-        for e in events:
-            if not e.cuda_event:  # torch creates the CUDA event lazily, on its first record
-                e.record()
-        arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
-        _check(_lib().lc_moe_forward_timed(*args, arr), "lc_moe_forward_timed")
+        _check(_lib().lc_moe_forward_timed(*args, _event_array(events)), "lc_moe_forward_timed")
+    return out
+
+
+def _event_array(events):
+    if len(events) != NUM_STAGES + 1:
+        raise ValueError(f"events: need {NUM_STAGES + 1} CUDA events")
+    for e in events:
+        if not e.cuda_event:  # torch creates the CUDA event lazily, on its first record
+            e.record()
+    return (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+
+
+def lc_moe_quantize_e4m3(src, dst=None, scale=None, stream=None):
+    """Row-wise E4M3 quantisation of a bf16 matrix [R, C] (any leading shape, rows = all but the
+    last dimension). Returns (codes uint8, same shape; scale float32 [R...])."""
+    if src.dtype != torch.bfloat16 or not src.is_cuda or not src.is_contiguous():
+        raise ValueError("src: expected a contiguous bf16 CUDA tensor")
+    C = src.shape[-1]
+    R = src.numel() // C if C else 0
+    if dst is None:
+        dst = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+    if scale is None:
+        scale = torch.empty(src.shape[:-1], dtype=torch.float32, device=src.device)
+    _need(dst, torch.uint8, tuple(src.shape), "dst")
+    _need(scale, torch.float32, tuple(src.shape[:-1]), "scale")
+    _check(_lib().lc_moe_quantize_e4m3(_ptr(src), R, C, _ptr(dst), _ptr(scale), _stream(stream)),
+           "lc_moe_quantize_e4m3")
+    return dst, scale
+
+
+def lc_moe_forward_fp8(x, wr, bias, w13q, w13_scale, w2, K: int, out=None, idx=None, gate=None,
+                       counts=None, ws=None, stream=None, events=None):
+    """MoE(x) with E4M3 gate/up projections: w13q [N, 2I, d] uint8 codes and w13_scale [N, 2I]
+    float32 (from lc_moe_quantize_e4m3); w2 [N, d, I] bf16. Returns ``out`` [T, d] bf16."""
+    T, d = x.shape
+    E = wr.shape[0]
+    N, two_i, _ = w13q.shape
+    I = two_i // 2
+    _need(x, torch.bfloat16, (T, d), "x")
+    _need(wr, torch.bfloat16, (E, d), "wr")
+    _need(bias, torch.float32, (E,), "bias")
+    _need(w13q, torch.uint8, (N, 2 * I, d), "w13q")
+    _need(w13_scale, torch.float32, (N, 2 * I), "w13_scale")
+    _need(w2, torch.bfloat16, (N, d, I), "w2")
+    if out is None:
+        out = torch.empty(T, d, dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, (T, d), "out")
+    if idx is not None:
+        _need(idx, torch.int32, (T, K), "idx")
+    if gate is not None:
+        _need(gate, torch.float32, (T, K), "gate")
+    if counts is not None:
+        _need(counts, torch.int32, (E,), "counts")
+    s = Shape(T, d, N, E - N, K, I)
+    if ws is None:
+        ws = new_workspace(s, OP_FORWARD_FP8, x.device)
+    args = [ctypes.byref(s), _ptr(x), _ptr(wr), _ptr(bias), _ptr(w13q), _ptr(w13_scale), _ptr(w2),
+            _ptr(out), _ptr(idx), _ptr(gate), _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)]
+    if events is None:
+        _check(_lib().lc_moe_forward_fp8(*args), "lc_moe_forward_fp8")
+    else:
+        _check(_lib().lc_moe_forward_fp8_timed(*args, _event_array(events)), "lc_moe_forward_fp8_timed")
     return out
 
 

@@ -37,11 +37,13 @@ int check_shape(const lc_moe_shape* s) {
 
 // Byte offsets of the forward workspace regions.
 struct FwdLayout {
-    size_t logits, idx, gate, offsets, row_token, pair_row, scratch, x_perm, h, y, total;
+    size_t logits, idx, gate, offsets, row_token, pair_row, scratch, xq, sx, s_row, x_perm, h, y, total;
     int64_t rows_cap;
 };
 
-FwdLayout fwd_layout(const lc_moe_shape* s) {
+// f8: the E4M3 variant (quantised token rows [T, d] bytes and their scales [T], grouped rows of
+// d bytes with their scales [rows_cap]); otherwise grouped rows of d bf16 values.
+FwdLayout fwd_layout(const lc_moe_shape* s, bool f8 = false) {
     FwdLayout L{};
     const size_t T = s->T, K = s->K, E = static_cast<size_t>(s->N) + s->Z;
     const int64_t rows_cap = static_cast<int64_t>(s->T) * (s->K < s->N ? s->K : s->N);
@@ -53,7 +55,12 @@ FwdLayout fwd_layout(const lc_moe_shape* s) {
     L.row_token = o; o = align_up(o + T * K * 4);
     L.pair_row = o;  o = align_up(o + T * K * 4);
     L.scratch = o;   o = align_up(o + permute_scratch_bytes(s->T, s->N));
-    L.x_perm = o;    o = align_up(o + static_cast<size_t>(rows_cap) * s->d * 2);
+    if (f8) {
+        L.xq = o;    o = align_up(o + T * s->d);
+        L.sx = o;    o = align_up(o + T * 4);
+        L.s_row = o; o = align_up(o + static_cast<size_t>(rows_cap) * 4);
+    }
+    L.x_perm = o;    o = align_up(o + static_cast<size_t>(rows_cap) * s->d * (f8 ? 1 : 2));
     L.h = o;         o = align_up(o + static_cast<size_t>(rows_cap) * s->I * 2);
     L.y = o;         o = align_up(o + static_cast<size_t>(rows_cap) * s->d * 2);
     L.total = o;
@@ -97,13 +104,18 @@ int record(void* const* events, int i, cudaStream_t st) {
 }
 
 int forward_impl(const lc_moe_shape* s, const void* x, const void* wr, const float* bias,
-                 const void* w13, const void* w2, void* out, int32_t* idx, float* gate,
-                 int32_t* counts, void* ws, size_t ws_bytes, void* stream, void* const* events) {
+                 const void* w13, const float* w13_scale, const void* w2, void* out, int32_t* idx,
+                 float* gate, int32_t* counts, void* ws, size_t ws_bytes, void* stream,
+                 void* const* events) {
+    // w13_scale != NULL selects the E4M3 experts (w13 then holds E4M3 codes)
+    const bool f8 = w13_scale != nullptr;
     LC_TRY(check_shape(s));
+    if (f8 && s->d % 128) return LC_MOE_ERR_UNSUPPORTED_SHAPE;
     if (!x || !wr || !bias || !w13 || !w2 || !out || !ws) return LC_MOE_ERR_INVALID_ARG;
-    const FwdLayout L = fwd_layout(s);
+    const FwdLayout L = fwd_layout(s, f8);
     if (ws_bytes < L.total) return LC_MOE_ERR_WORKSPACE_TOO_SMALL;
-    for (const void* p : {x, wr, static_cast<const void*>(bias), w13, w2, static_cast<const void*>(out),
+    for (const void* p : {x, wr, static_cast<const void*>(bias), w13, static_cast<const void*>(w13_scale), w2,
+                          static_cast<const void*>(out),
                           static_cast<const void*>(idx), static_cast<const void*>(gate),
                           static_cast<const void*>(counts), static_cast<const void*>(ws)})
         if (p && !aligned16(p)) return LC_MOE_ERR_MISALIGNED;
@@ -130,9 +142,21 @@ int forward_impl(const lc_moe_shape* s, const void* x, const void* wr, const flo
     LC_TRY(record(events, LC_MOE_STAGE_PERMUTE, st));
     LC_CUDA(launch_permute(idx_w, s->T, s->K, s->N, E, offsets, row_token, pair_row, scratch, status, st));
     LC_TRY(record(events, LC_MOE_STAGE_GATHER, st));
-    LC_CUDA(launch_gather(x, s->T, s->d, s->K, pair_row, x_perm, st));
-    LC_TRY(record(events, LC_MOE_STAGE_GEMM1, st));
-    LC_CUDA(launch_grouped_swiglu(x_perm, L.rows_cap, offsets, s->N, w13, s->d, s->I, h, status, st));
+    if (f8) {
+        // quantise each token row once, then copy codes and scale to each of its FFN rows
+        void* xq = at<void>(ws, L.xq);
+        float* sx = at<float>(ws, L.sx);
+        float* s_row = at<float>(ws, L.s_row);
+        LC_CUDA(launch_quantize_rows_e4m3(x, s->T, s->d, xq, sx, st));
+        LC_CUDA(launch_gather_e4m3(xq, sx, s->T, s->d, s->K, pair_row, x_perm, s_row, st));
+        LC_TRY(record(events, LC_MOE_STAGE_GEMM1, st));
+        LC_CUDA(launch_grouped_swiglu_e4m3(x_perm, s_row, L.rows_cap, offsets, s->N, w13, w13_scale, s->d,
+                                           s->I, h, status, st));
+    } else {
+        LC_CUDA(launch_gather(x, s->T, s->d, s->K, pair_row, x_perm, st));
+        LC_TRY(record(events, LC_MOE_STAGE_GEMM1, st));
+        LC_CUDA(launch_grouped_swiglu(x_perm, L.rows_cap, offsets, s->N, w13, s->d, s->I, h, status, st));
+    }
     LC_TRY(record(events, LC_MOE_STAGE_GEMM2, st));
     LC_CUDA(launch_grouped_down(h, L.rows_cap, offsets, s->N, w2, s->d, s->I, y, status, st));
     LC_TRY(record(events, LC_MOE_STAGE_COMBINE, st));
@@ -192,6 +216,7 @@ size_t lc_moe_workspace_bytes(const lc_moe_shape* s, int op) {
     if (check_shape(s) != LC_MOE_OK) return 0;
     switch (op) {
         case LC_MOE_OP_FORWARD: return fwd_layout(s).total;
+        case LC_MOE_OP_FORWARD_FP8: return s->d % 128 ? 0 : fwd_layout(s, true).total;
         case LC_MOE_OP_ROUTE: return route_ws_bytes(s);
         case LC_MOE_OP_PERMUTE: return permute_ws_bytes(s);
         case LC_MOE_OP_STATUS: return kStatusBytes;
@@ -207,7 +232,8 @@ void lc_moe_set_wait_limit_ns(uint64_t limit_ns) {
 int lc_moe_forward(const lc_moe_shape* s, const void* x, const void* wr, const float* bias,
                    const void* w13, const void* w2, void* out, int32_t* idx, float* gate,
                    int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
-    return forward_impl(s, x, wr, bias, w13, w2, out, idx, gate, counts, ws, ws_bytes, stream, nullptr);
+    return forward_impl(s, x, wr, bias, w13, nullptr, w2, out, idx, gate, counts, ws, ws_bytes, stream,
+                        nullptr);
 }
 
 int lc_moe_forward_timed(const lc_moe_shape* s, const void* x, const void* wr, const float* bias,
@@ -217,7 +243,40 @@ int lc_moe_forward_timed(const lc_moe_shape* s, const void* x, const void* wr, c
     if (!events) return LC_MOE_ERR_INVALID_ARG;
     for (int i = 0; i <= LC_MOE_NUM_STAGES; ++i)
         if (!events[i]) return LC_MOE_ERR_INVALID_ARG;
-    return forward_impl(s, x, wr, bias, w13, w2, out, idx, gate, counts, ws, ws_bytes, stream, events);
+    return forward_impl(s, x, wr, bias, w13, nullptr, w2, out, idx, gate, counts, ws, ws_bytes, stream,
+                        events);
+}
+
+int lc_moe_forward_fp8(const lc_moe_shape* s, const void* x, const void* wr, const float* bias,
+                       const void* w13q, const float* w13_scale, const void* w2, void* out,
+                       int32_t* idx, float* gate, int32_t* counts, void* ws, size_t ws_bytes,
+                       void* stream) {
+    if (!w13_scale) return LC_MOE_ERR_INVALID_ARG;
+    return forward_impl(s, x, wr, bias, w13q, w13_scale, w2, out, idx, gate, counts, ws, ws_bytes,
+                        stream, nullptr);
+}
+
+int lc_moe_forward_fp8_timed(const lc_moe_shape* s, const void* x, const void* wr, const float* bias,
+                             const void* w13q, const float* w13_scale, const void* w2, void* out,
+                             int32_t* idx, float* gate, int32_t* counts, void* ws, size_t ws_bytes,
+                             void* stream, void* const* events) {
+    if (!w13_scale || !events) return LC_MOE_ERR_INVALID_ARG;
+    for (int i = 0; i <= LC_MOE_NUM_STAGES; ++i)
+        if (!events[i]) return LC_MOE_ERR_INVALID_ARG;
+    return forward_impl(s, x, wr, bias, w13q, w13_scale, w2, out, idx, gate, counts, ws, ws_bytes,
+                        stream, events);
+}
+
+int lc_moe_quantize_e4m3(const void* src, int64_t rows, int32_t cols, void* dst, float* scale,
+                         void* stream) {
+    if (rows < 0 || cols < 8 || cols % 8) return LC_MOE_ERR_INVALID_ARG;
+    if (rows == 0) return LC_MOE_OK;
+    if (!src || !dst || !scale) return LC_MOE_ERR_INVALID_ARG;
+    if (!aligned16(src) || !aligned16(dst) || (reinterpret_cast<uintptr_t>(scale) & 3u))
+        return LC_MOE_ERR_MISALIGNED;
+    LC_TRY(device_ok());
+    LC_CUDA(launch_quantize_rows_e4m3(src, rows, cols, dst, scale, static_cast<cudaStream_t>(stream)));
+    return LC_MOE_OK;
 }
 
 int lc_moe_route(const lc_moe_shape* s, const void* x, const void* wr, const float* bias,

@@ -153,6 +153,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor, kind::f8f6f4: A and B E4M3 (format code 0), K-major; D fp32; M x N.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+    return (1u << 4)                                   // D format: f32
+           | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, one 128 x N x 16 step, issued by a single thread.
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                           uint32_t idesc, uint32_t accumulate) {
@@ -255,6 +262,19 @@ __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, 
         : "memory");
 }
 
+// As umma_bf16_pair with E4M3 operands: one 256 x N x 32 step (32 bytes of K per operand row).
+__device__ __forceinline__ void umma_e4m3_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n"
+        ".reg .pred p;\n"
+        "setp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n"
+        "}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive once on the mbarrier at the same offset in every CTA of `cta_mask` when every tcgen05
 // operation issued so far by this thread has completed.
 __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
@@ -288,6 +308,8 @@ uint64_t wait_limit_ns();
 
 // Row-major bf16 matrix [rows, cols] as a TMA map with 64 x box_rows boxes and the 128-byte swizzle.
 bool make_tma_map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// Same for a row-major byte matrix (E4M3 codes) [rows, cols]: boxes of 128 bytes x box_rows.
+bool make_tma_map_2d_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
 // Router GEMM: logits[T, E] fp32 = x[T, d] * wr[E, d]^T.
 cudaError_t launch_router_gemm(const void* x, const void* wr, float* logits, int T, int d, int E,
@@ -319,6 +341,23 @@ cudaError_t launch_permute(const int32_t* idx, int T, int K, int N, int E, int32
                            uint32_t* status, cudaStream_t st);
 cudaError_t launch_gather(const void* x, int T, int d, int K, const int32_t* pair_row,
                           void* x_perm, cudaStream_t st);
+// Row gather of E4M3 token rows (d bytes each) with their scales: x_perm[pair_row[t,k]] = xq[t],
+// s_row[pair_row[t,k]] = sx[t].
+cudaError_t launch_gather_e4m3(const void* xq, const float* sx, int T, int d, int K,
+                               const int32_t* pair_row, void* x_perm, float* s_row, cudaStream_t st);
+
+// Row-wise E4M3 quantisation of a bf16 matrix [R, C] (C % 8 == 0): scale[r] = amax / 448
+// (1 for an all-zero row), dst[r, c] = E4M3(src[r, c] / scale[r]) (round to nearest even,
+// saturating at 448).
+cudaError_t launch_quantize_rows_e4m3(const void* src, int64_t R, int C, void* dst, float* scale,
+                                      cudaStream_t st);
+
+// Grouped GEMM 1 on E4M3 operands: rows x_perm [rows_cap, d] (codes) with row scales s_row,
+// W13 codes [N, 2I, d] with one scale per weight row; the SwiGLU epilogue applies both scales.
+cudaError_t launch_grouped_swiglu_e4m3(const void* x_perm, const float* s_row, int64_t rows_cap,
+                                       const int32_t* offsets, int N, const void* w13q,
+                                       const float* w13_scale, int d, int I, void* h,
+                                       uint32_t* status, cudaStream_t st);
 // Grouping with its tables in a file-scope device array (no caller workspace).
 bool permute_noalloc_fits(int T, int N);
 cudaError_t launch_permute_noalloc(const int32_t* idx, int T, int K, int N, int E, int32_t* offsets,

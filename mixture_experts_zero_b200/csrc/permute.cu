@@ -156,13 +156,14 @@ constexpr int GATHER_THREADS = 256;
 
 __global__ void __launch_bounds__(GATHER_THREADS)
     gather_kernel(const uint4* __restrict__ x, int T, int d8, int K, const int32_t* __restrict__ pair_row,
-                  uint4* __restrict__ x_perm) {
+                  uint4* __restrict__ x_perm, const float* __restrict__ sx, float* __restrict__ s_row) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (GATHER_THREADS / 32);
     for (int t = blockIdx.x * (GATHER_THREADS / 32) + warp; t < T; t += warps_total) {
         const int my_row = (lane < K) ? pair_row[static_cast<int64_t>(t) * K + lane] : -1;
         const uint32_t dests = __ballot_sync(0xffffffffu, my_row >= 0);
         if (!dests) continue;
+        if (s_row && my_row >= 0) s_row[my_row] = sx[t];  // row scale of E4M3 rows
         const uint4* src = x + static_cast<int64_t>(t) * d8;
         for (int c0 = 0; c0 < d8; c0 += 128) {  // warp-uniform trip count; 4 loads in flight
             uint4 v[4];
@@ -235,7 +236,20 @@ cudaError_t launch_gather(const void* x, int T, int d, int K, const int32_t* pai
     int blocks = (T + warps - 1) / warps;
     if (blocks > di->sm_count * 8) blocks = di->sm_count * 8;
     gather_kernel<<<blocks, GATHER_THREADS, 0, st>>>(static_cast<const uint4*>(x), T, d / 8, K, pair_row,
-                                                      static_cast<uint4*>(x_perm));
+                                                      static_cast<uint4*>(x_perm), nullptr, nullptr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_e4m3(const void* xq, const float* sx, int T, int d, int K,
+                               const int32_t* pair_row, void* x_perm, float* s_row, cudaStream_t st) {
+    const DevInfo* di = current_device_info();
+    if (!di) return cudaErrorUnknown;
+    if (T == 0) return cudaSuccess;
+    const int warps = GATHER_THREADS / 32;
+    int blocks = (T + warps - 1) / warps;
+    if (blocks > di->sm_count * 8) blocks = di->sm_count * 8;
+    gather_kernel<<<blocks, GATHER_THREADS, 0, st>>>(static_cast<const uint4*>(xq), T, d / 16, K, pair_row,
+                                                      static_cast<uint4*>(x_perm), sx, s_row);
     return cudaGetLastError();
 }
 

@@ -266,6 +266,19 @@ bool make_tma_map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t co
     return r == CUDA_SUCCESS;
 }
 
+bool make_tma_map_2d_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 cudaError_t launch_router_gemm(const void* x, const void* wr, float* logits, int T, int d, int E,
                                uint32_t* status, cudaStream_t st) {
     const DevInfo* di = current_device_info();

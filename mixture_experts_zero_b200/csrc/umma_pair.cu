@@ -78,6 +78,8 @@ struct PairArgs {
     int cold_rows;           // experts with 0 < rows < cold_rows use weight tiles only
     int rem_rows;            // an expert's rows past its last full 256-row tile: fewer than this
                              // run as weight tiles, otherwise as one more row tile
+    const float* row_scale;  // E4M3 GEMM 1: scale of each grouped row [rows_cap]
+    const float* w_scale;    // E4M3 GEMM 1: scale of each weight row [n_groups * b_group_rows]
 };
 
 // Epilogue transpose tile of one warp: 32 rows x 32 features (bf16), 64 bytes per row, its four
@@ -114,6 +116,13 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint6
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
 
+template <bool F8>
+__device__ __forceinline__ void mma_step(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    if (F8) umma_e4m3_pair(d_tmem, adesc, bdesc, idesc, accumulate);
+    else umma_bf16_pair(d_tmem, adesc, bdesc, idesc, accumulate);
+}
+
 __device__ __forceinline__ int upper_group(const int32_t* pre, int n, int v) {
     int lo = 0, hi = n - 1;
     while (lo < hi) {
@@ -124,7 +133,10 @@ __device__ __forceinline__ int upper_group(const int32_t* pre, int n, int v) {
     return lo;
 }
 
-template <int MODE>
+// F8: operands are E4M3 codes (GEMM 1 only): a 128-byte k-step holds 128 elements, the MMAs are
+// kind::f8f6f4 (K = 32 per instruction), and the epilogue multiplies each accumulator by its row's
+// scale and its weight row's scale before the SwiGLU.
+template <int MODE, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     umma_pair_kernel(const __grid_constant__ CUtensorMap mapRows, const __grid_constant__ CUtensorMap mapW,
                      const __grid_constant__ CUtensorMap mapTok, const PairArgs g) {
@@ -223,7 +235,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const int total_r = rpre_s[g.n_groups];
     const int total_s = spre_s[g.n_groups];
     const int total = total_r + total_s;
-    const int nk = g.kdim / BK;
+    constexpr int KB = F8 ? 2 * BK : BK;  // elements per 128-byte k-step
+    const int nk = g.kdim / KB;
 
     auto decode = [&](int tile) {
         Tile tl;
@@ -288,7 +301,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 uint8_t* sb = sa + A_BYTES;
                 const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
                 if (leader) mbar_arrive_expect_tx(&full[s], 2 * cta_bytes);
-                const int kx = kb * BK;
+                const int kx = kb * KB;
                 if (!tl.swap) {
                     tma_load_2d_pair(sa, &mapRows, bar, kx, static_cast<int32_t>(tl.row0 + rank * HALF_M), pol_normal);
                     // GEMM 1: leader gate rows, peer up rows; GEMM 2: 128 output features each
@@ -334,7 +347,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         bool ok = true;
         for (int tile = cluster; tile < total && ok; tile += n_clusters) {
             const Tile tl = decode(tile);
-            const uint32_t idesc = idesc_bf16_f32(2 * HALF_M, tl.swap ? tl.ntok : 2 * HALF_M);
+            const uint32_t idesc = F8 ? idesc_e4m3_f32(2 * HALF_M, tl.swap ? tl.ntok : 2 * HALF_M)
+                                      : idesc_bf16_f32(2 * HALF_M, tl.swap ? tl.ntok : 2 * HALF_M);
             if (!mbar_wait(&tempty[acc], aph ^ 1u, g.wait_ns, abort_flag, g.status)) {
                 ok = false;
                 break;
@@ -354,13 +368,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     const uint64_t td = sw128_kmajor_desc(smem_u32(sa + 2 * A_BYTES));
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        umma_bf16_pair(d_tmem, ad + 2 * kk, td + 2 * kk, idesc, (kb | kk) != 0);
-                        umma_bf16_pair(d_tmem + 128, bd + 2 * kk, td + 2 * kk, idesc, (kb | kk) != 0);
+                        mma_step<F8>(d_tmem, ad + 2 * kk, td + 2 * kk, idesc, (kb | kk) != 0);
+                        mma_step<F8>(d_tmem + 128, bd + 2 * kk, td + 2 * kk, idesc, (kb | kk) != 0);
                     }
                 } else {
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        umma_bf16_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                        mma_step<F8>(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
                 }
                 umma_commit_pair(&empty[s], 0x3);
                 if (++s == STAGES) {
@@ -400,6 +414,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         tmem_ld_wait();
                         const int f0 = tl.n0 + c;
                         if (valid && f0 < g.n_out) {
+                            if (F8) {
+                                // (acc * row scale) * weight-row scale, gate and up separately
+                                const float sr = __ldg(g.row_scale + grow);
+                                const float4* sg4 = reinterpret_cast<const float4*>(
+                                    g.w_scale + static_cast<int64_t>(tl.grp) * g.b_group_rows + f0);
+                                const float4* su4 = reinterpret_cast<const float4*>(
+                                    g.w_scale + static_cast<int64_t>(tl.grp) * g.b_group_rows + g.up_off + f0);
+#pragma unroll
+                                for (int j4 = 0; j4 < 8; ++j4) {
+                                    const float4 a = __ldg(sg4 + j4), b = __ldg(su4 + j4);
+                                    const float sa[4] = {a.x, a.y, a.z, a.w}, sb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                                    for (int u = 0; u < 4; ++u) {
+                                        gv[4 * j4 + u] = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(gv[4 * j4 + u]), sr), sa[u]));
+                                        uv[4 * j4 + u] = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(uv[4 * j4 + u]), sr), sb[u]));
+                                    }
+                                }
+                            }
                             uint32_t pk[16];
 #pragma unroll
                             for (int j = 0; j < 16; ++j)
@@ -442,6 +474,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         uint32_t uv[32];
                         tmem_ld_32x32b_x32(tb + HALF_M + c0, uv);
                         tmem_ld_wait();
+                        if (F8) {
+                            // lane = weight row (feature), column j = grouped row c0 + j
+                            const int64_t wb = static_cast<int64_t>(tl.grp) * g.b_group_rows;
+                            const int fl = f0 + lane < g.n_out ? f0 + lane : g.n_out - 1;
+                            const float sg = __ldg(g.w_scale + wb + fl);
+                            const float su = __ldg(g.w_scale + wb + g.up_off + fl);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                int64_t rr = tl.row0 + c0 + j;
+                                if (rr >= g.rows_cap) rr = g.rows_cap - 1;
+                                const float sr = __ldg(g.row_scale + rr);
+                                v[j] = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(v[j]), sr), sg));
+                                uv[j] = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(uv[j]), sr), su));
+                            }
+                        }
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
                             v[j] = __float_as_uint(silu_mul(__uint_as_float(v[j]), __uint_as_float(uv[j])));
@@ -483,7 +530,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     }
 }
 
-template <int MODE>
+template <int MODE, bool F8>
 cudaError_t launch_pair(const CUtensorMap& mr, const CUtensorMap& mw, const CUtensorMap& mt,
                         const PairArgs& args, int grid, cudaStream_t st) {
     const size_t smem = Layout::bytes(args.n_groups);
@@ -496,11 +543,11 @@ cudaError_t launch_pair(const CUtensorMap& mr, const CUtensorMap& mw, const CUte
         e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         if (e != cudaSuccess) return e;
         if (static_cast<int>(smem) > max_optin) return cudaErrorInvalidValue;
-        e = cudaFuncSetAttribute(umma_pair_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_optin);
+        e = cudaFuncSetAttribute(umma_pair_kernel<MODE, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_optin);
         if (e != cudaSuccess) return e;
         configured[dev] = max_optin;
     }
-    umma_pair_kernel<MODE><<<grid, NUM_THREADS, smem, st>>>(mr, mw, mt, args);
+    umma_pair_kernel<MODE, F8><<<grid, NUM_THREADS, smem, st>>>(mr, mw, mt, args);
     return cudaGetLastError();
 }
 
@@ -508,15 +555,10 @@ int pair_grid(const DevInfo* di) { return (di->sm_count / 2) * 2; }
 
 }  // namespace
 
-cudaError_t launch_grouped_swiglu(const void* x_perm, int64_t rows_cap, const int32_t* offsets,
-                                  int N, const void* w13, int d, int I, void* h, uint32_t* status,
-                                  cudaStream_t st) {
-    const DevInfo* di = current_device_info();
-    if (!di) return cudaErrorUnknown;
-    CUtensorMap mr, mw, mt;
-    if (!make_tma_map_2d(&mr, x_perm, static_cast<uint64_t>(rows_cap), d, HALF_M)) return cudaErrorInvalidValue;
-    if (!make_tma_map_2d(&mw, w13, static_cast<uint64_t>(N) * 2 * I, d, HALF_M)) return cudaErrorInvalidValue;
-    if (!make_tma_map_2d(&mt, x_perm, static_cast<uint64_t>(rows_cap), d, TOK_BOX)) return cudaErrorInvalidValue;
+namespace {
+
+PairArgs swiglu_args(int64_t rows_cap, const int32_t* offsets, int N, int d, int I, void* h,
+                     uint32_t* status) {
     PairArgs a{};
     a.offsets = offsets;
     a.out = static_cast<__nv_bfloat16*>(h);
@@ -535,7 +577,38 @@ cudaError_t launch_grouped_swiglu(const void* x_perm, int64_t rows_cap, const in
     // weight-tile N <= 128 keeps gate and up in one 256-column accumulator
     a.cold_rows = 128;
     a.rem_rows = 128;
-    return launch_pair<MODE_SWIGLU>(mr, mw, mt, a, pair_grid(di), st);
+    return a;
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_swiglu(const void* x_perm, int64_t rows_cap, const int32_t* offsets,
+                                  int N, const void* w13, int d, int I, void* h, uint32_t* status,
+                                  cudaStream_t st) {
+    const DevInfo* di = current_device_info();
+    if (!di) return cudaErrorUnknown;
+    CUtensorMap mr, mw, mt;
+    if (!make_tma_map_2d(&mr, x_perm, static_cast<uint64_t>(rows_cap), d, HALF_M)) return cudaErrorInvalidValue;
+    if (!make_tma_map_2d(&mw, w13, static_cast<uint64_t>(N) * 2 * I, d, HALF_M)) return cudaErrorInvalidValue;
+    if (!make_tma_map_2d(&mt, x_perm, static_cast<uint64_t>(rows_cap), d, TOK_BOX)) return cudaErrorInvalidValue;
+    const PairArgs a = swiglu_args(rows_cap, offsets, N, d, I, h, status);
+    return launch_pair<MODE_SWIGLU, false>(mr, mw, mt, a, pair_grid(di), st);
+}
+
+cudaError_t launch_grouped_swiglu_e4m3(const void* x_perm, const float* s_row, int64_t rows_cap,
+                                       const int32_t* offsets, int N, const void* w13q,
+                                       const float* w13_scale, int d, int I, void* h,
+                                       uint32_t* status, cudaStream_t st) {
+    const DevInfo* di = current_device_info();
+    if (!di) return cudaErrorUnknown;
+    CUtensorMap mr, mw, mt;
+    if (!make_tma_map_2d_u8(&mr, x_perm, static_cast<uint64_t>(rows_cap), d, HALF_M)) return cudaErrorInvalidValue;
+    if (!make_tma_map_2d_u8(&mw, w13q, static_cast<uint64_t>(N) * 2 * I, d, HALF_M)) return cudaErrorInvalidValue;
+    if (!make_tma_map_2d_u8(&mt, x_perm, static_cast<uint64_t>(rows_cap), d, TOK_BOX)) return cudaErrorInvalidValue;
+    PairArgs a = swiglu_args(rows_cap, offsets, N, d, I, h, status);
+    a.row_scale = s_row;
+    a.w_scale = w13_scale;
+    return launch_pair<MODE_SWIGLU, true>(mr, mw, mt, a, pair_grid(di), st);
 }
 
 cudaError_t launch_grouped_down(const void* h, int64_t rows_cap, const int32_t* offsets, int N,
@@ -564,7 +637,7 @@ cudaError_t launch_grouped_down(const void* h, int64_t rows_cap, const int32_t* 
     a.s_tiles = (d + 2 * HALF_M - 1) / (2 * HALF_M);
     a.cold_rows = 256;
     a.rem_rows = 256;
-    return launch_pair<MODE_DOWN>(mr, mw, mt, a, pair_grid(di), st);
+    return launch_pair<MODE_DOWN, false>(mr, mw, mt, a, pair_grid(di), st);
 }
 
 }  // namespace lcmoe
