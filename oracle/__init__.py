@@ -50,8 +50,9 @@ def configure(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oracle_float_to_e4m3.argtypes = [ctypes.c_float]
     L.oracle_float_to_e4m3.restype = ctypes.c_uint8
     L.oracle_quantize_rows_e4m3.argtypes = [P, I64, I64, P, P]
-    L.oracle_expert_rows_fp8.argtypes = [P, P, P, I64, I64, I64, P, P, P, P, P]
-    L.oracle_forward_fp8.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, P, P, P, P, P, P]
+    L.oracle_expert_rows_fp8.argtypes = [P, P, P, I64, I64, I64, P, P, P, P, P, P]
+    L.oracle_expert_down_fp8.argtypes = [P, P, I64, I64, I64, P, P, P]
+    L.oracle_forward_fp8.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I64, I64, I64, P, P, P, P, P, P]
     L.oracle_forward_fp8.restype = I64
     return L
 
@@ -257,42 +258,62 @@ def quantize_rows_e4m3(src: np.ndarray):
 
 
 def expert_rows_fp8(xq: np.ndarray, sx: np.ndarray, row_expert: np.ndarray, w13q: np.ndarray,
-                    w13_scale: np.ndarray, w2: np.ndarray, want_h: bool = True):
-    """FP8 SwiGLU expert of each row: gate/up from E4M3 codes with row scales, down in bf16.
-    w13q is [N, 2I, d] uint8 with w13_scale [N, 2I]; w2 is [N, d, I] bf16 bits."""
+                    w13_scale: np.ndarray, w2q: np.ndarray, w2_scale: np.ndarray,
+                    want_h: bool = True):
+    """FP8 SwiGLU expert of each row: gate/up from E4M3 codes with row scales, H rounded to bf16,
+    then H quantised per row and the down projection from E4M3 codes. w13q [N, 2I, d] uint8 with
+    w13_scale [N, 2I]; w2q [N, d, I] uint8 with w2_scale [N, d]. Returns (H, Y) bf16 bits."""
     xq = _c(xq, np.uint8); sx = _c(sx, np.float32); row_expert = _c(row_expert, np.int32)
-    w13q = _c(w13q, np.uint8); w13_scale = _c(w13_scale, np.float32); w2 = _c(w2, np.uint16)
+    w13q = _c(w13q, np.uint8); w13_scale = _c(w13_scale, np.float32)
+    w2q = _c(w2q, np.uint8); w2_scale = _c(w2_scale, np.float32)
     M, d = xq.shape
     n, two_i, d2 = w13q.shape
     I = two_i // 2
-    assert d2 == d and w2.shape == (n, d, I) and w13_scale.shape == (n, two_i)
-    assert sx.shape == (M,) and row_expert.shape == (M,)
+    assert d2 == d and w2q.shape == (n, d, I) and w13_scale.shape == (n, two_i)
+    assert w2_scale.shape == (n, d) and sx.shape == (M,) and row_expert.shape == (M,)
     if M and (row_expert.min() < 0 or row_expert.max() >= n):
         raise ValueError("row_expert out of range")
     h = np.empty((M, I), dtype=np.uint16) if want_h else None
     y = np.empty((M, d), dtype=np.uint16)
     lib().oracle_expert_rows_fp8(_p(xq), _p(sx), _p(row_expert), M, d, I, _p(w13q), _p(w13_scale),
-                                 _p(w2), _p(h), _p(y))
+                                 _p(w2q), _p(w2_scale), _p(h), _p(y))
     return h, y
 
 
-def forward_fp8(x, wr, bias, w13q, w13_scale, w2, N: int, Z: int, K: int,
+def expert_down_fp8(h: np.ndarray, row_expert: np.ndarray, w2q: np.ndarray, w2_scale: np.ndarray):
+    """The FP8 down projection alone: each bf16 row of H quantised per row, Y = bf16 of the
+    scaled E4M3 product with W2 codes w2q [N, d, I] and scales w2_scale [N, d]."""
+    h = _c(h, np.uint16); row_expert = _c(row_expert, np.int32)
+    w2q = _c(w2q, np.uint8); w2_scale = _c(w2_scale, np.float32)
+    M, I = h.shape
+    n, d, I2 = w2q.shape
+    assert I2 == I and w2_scale.shape == (n, d) and row_expert.shape == (M,)
+    if M and (row_expert.min() < 0 or row_expert.max() >= n):
+        raise ValueError("row_expert out of range")
+    y = np.empty((M, d), dtype=np.uint16)
+    lib().oracle_expert_down_fp8(_p(h), _p(row_expert), M, d, I, _p(w2q), _p(w2_scale), _p(y))
+    return y
+
+
+def forward_fp8(x, wr, bias, w13q, w13_scale, w2q, w2_scale, N: int, Z: int, K: int,
                 counts: np.ndarray | None = None):
-    """The layer with FP8 gate/up projections (token rows quantised per row). Same return
-    value as ``forward``."""
+    """The layer with FP8 experts (token rows and H rows quantised per row). Same return value
+    as ``forward``."""
     x = _c(x, np.uint16); wr = _c(wr, np.uint16); bias = _c(bias, np.float32)
-    w13q = _c(w13q, np.uint8); w13_scale = _c(w13_scale, np.float32); w2 = _c(w2, np.uint16)
+    w13q = _c(w13q, np.uint8); w13_scale = _c(w13_scale, np.float32)
+    w2q = _c(w2q, np.uint8); w2_scale = _c(w2_scale, np.float32)
     T, d = x.shape
     E = N + Z
-    I = w2.shape[2]
-    assert wr.shape == (E, d) and w13q.shape == (N, 2 * I, d) and w2.shape == (N, d, I)
-    assert w13_scale.shape == (N, 2 * I)
+    I = w2q.shape[2]
+    assert wr.shape == (E, d) and w13q.shape == (N, 2 * I, d) and w2q.shape == (N, d, I)
+    assert w13_scale.shape == (N, 2 * I) and w2_scale.shape == (N, d)
     out = np.empty((T, d), dtype=np.uint16)
     logits = np.empty((T, E), dtype=np.float32)
     idx = np.empty((T, K), dtype=np.int32)
     gate = np.empty((T, K), dtype=np.float32)
     cnt = np.zeros(E, dtype=np.int32) if counts is None else _c(counts, np.int32)
     acc = np.empty((T, d), dtype=np.float64)
-    bad = lib().oracle_forward_fp8(_p(x), _p(wr), _p(bias), _p(w13q), _p(w13_scale), _p(w2), T, d,
-                                   N, Z, K, I, _p(out), _p(logits), _p(idx), _p(gate), _p(cnt), _p(acc))
+    bad = lib().oracle_forward_fp8(_p(x), _p(wr), _p(bias), _p(w13q), _p(w13_scale), _p(w2q),
+                                   _p(w2_scale), T, d, N, Z, K, I, _p(out), _p(logits), _p(idx),
+                                   _p(gate), _p(cnt), _p(acc))
     return dict(out=out, out_exact=acc, logits=logits, idx=idx, gate=gate, counts=cnt, bad=int(bad))

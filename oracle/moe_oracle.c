@@ -374,8 +374,8 @@ int64_t oracle_forward(const uint16_t* x, const uint16_t* wr, const float* bias,
 /* FP8 experts. The LongCat-Flash llm-wiki entity page, section 5 (inference and deployment),   */
 /* lists FP8/BF16 quantisation among the system-level optimisations and an FP8 deployment on   */
 /* one node in its measured-performance table; it gives no scaling scheme. Reading used here:  */
-/* the gate and up projections run on E4M3 operands, each weight row (output feature) and each */
-/* token row carrying one fp32 scale (amax / 448); the down projection stays bf16.             */
+/* all three expert projections run on E4M3 operands, each weight row (output feature) and    */
+/* each activation row (a token row of x, a row of H) carrying one fp32 scale (amax / 448).    */
 /*                                                                                              */
 /* E4M3 as the OCP 8-bit floating point format defines it: sign, 4 exponent bits (bias 7),      */
 /* 3 mantissa bits; exponent field 0 holds subnormals m * 2^-9; S.1111.111 is NaN; there is no  */
@@ -435,13 +435,43 @@ void oracle_quantize_rows_e4m3(const uint16_t* src, int64_t R, int64_t C, uint8_
     }
 }
 
+/* FP8 down projection of given bf16 rows H [M, I]: each row is quantised like any other row
+ * (oracle_quantize_rows_e4m3), W2q[e] holds the codes of Wd [d, I] with one scale per output
+ * feature in w2_scale[e * d + i]:
+ *   Y_i = bf16( sum_j (sh qh_j) (sw_i qw_ij) )   (double). */
+static void down_row_fp8(const uint16_t* hrow, int64_t I, const uint8_t* w2q, const float* w2s,
+                         int64_t d, uint16_t* yrow) {
+    uint8_t* hq = (uint8_t*)malloc((size_t)I);
+    float sh;
+    oracle_quantize_rows_e4m3(hrow, 1, I, hq, &sh);
+    double* hd = (double*)malloc((size_t)I * sizeof(double));
+    for (int64_t j = 0; j < I; ++j) hd[j] = (double)sh * oracle_e4m3_to_double(hq[j]);
+    for (int64_t i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int64_t j = 0; j < I; ++j) acc += hd[j] * ((double)w2s[i] * oracle_e4m3_to_double(w2q[i * I + j]));
+        yrow[i] = oracle_double_to_bf16(acc);
+    }
+    free(hq); free(hd);
+}
+
+void oracle_expert_down_fp8(const uint16_t* h, const int32_t* row_expert, int64_t M, int64_t d,
+                            int64_t I, const uint8_t* w2q, const float* w2_scale, uint16_t* y) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < M; ++r) {
+        const int64_t e = row_expert[r];
+        down_row_fp8(h + r * I, I, w2q + e * d * I, w2_scale + e * d, d, y + r * d);
+    }
+}
+
 /* FP8 experts on grouped rows: row r holds the E4M3 codes xq[r, :] of its token with scale
- * sx[r]; W13q[e] = [Wg; Wu] codes [2I, d] with one scale per row in w13_scale[e * 2I + j].
+ * sx[r]; W13q[e] = [Wg; Wu] codes [2I, d] with one scale per row in w13_scale[e * 2I + j];
+ * W2q[e] codes [d, I] with one scale per row in w2_scale[e * d + i].
  *   G_j = sum_k (sx qx_k) (sg_j qg_jk),  U_j likewise   (double)
- *   H_j = bf16( G_j sigmoid(G_j) U_j ),  Y = bf16( H Wd[e]^T )  (Wd bf16, as in step 7). */
+ *   H_j = bf16( G_j sigmoid(G_j) U_j ),  then the FP8 down projection of H above. */
 void oracle_expert_rows_fp8(const uint8_t* xq, const float* sx, const int32_t* row_expert,
                             int64_t M, int64_t d, int64_t I, const uint8_t* w13q,
-                            const float* w13_scale, const uint16_t* w2, uint16_t* h, uint16_t* y) {
+                            const float* w13_scale, const uint8_t* w2q, const float* w2_scale,
+                            uint16_t* h, uint16_t* y) {
     #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t r = 0; r < M; ++r) {
         const int64_t e = row_expert[r];
@@ -450,7 +480,7 @@ void oracle_expert_rows_fp8(const uint8_t* xq, const float* sx, const int32_t* r
         const float* sg = w13_scale + e * 2 * I;
         const float* su = sg + I;
         double* xd = (double*)malloc((size_t)d * sizeof(double));
-        double* hd = (double*)malloc((size_t)I * sizeof(double));
+        uint16_t* hrow = (uint16_t*)malloc((size_t)I * sizeof(uint16_t));
         for (int64_t k = 0; k < d; ++k) xd[k] = (double)sx[r] * oracle_e4m3_to_double(xq[r * d + k]);
         for (int64_t j = 0; j < I; ++j) {
             double G = 0.0, U = 0.0;
@@ -459,12 +489,11 @@ void oracle_expert_rows_fp8(const uint8_t* xq, const float* sx, const int32_t* r
                 U += xd[k] * ((double)su[j] * oracle_e4m3_to_double(wu[j * d + k]));
             }
             const double silu = G / (1.0 + exp(-G));
-            uint16_t hb = oracle_double_to_bf16(silu * U);
-            if (h) h[r * I + j] = hb;
-            hd[j] = bf16_to_double(hb);
+            hrow[j] = oracle_double_to_bf16(silu * U);
+            if (h) h[r * I + j] = hrow[j];
         }
-        down_row(hd, w2 + e * d * I, d, I, y + r * d);
-        free(xd); free(hd);
+        down_row_fp8(hrow, I, w2q + e * d * I, w2_scale + e * d, d, y + r * d);
+        free(xd); free(hrow);
     }
 }
 
@@ -472,10 +501,10 @@ void oracle_expert_rows_fp8(const uint8_t* xq, const float* sx, const int32_t* r
  * oracle_quantize_rows_e4m3 and every FFN pick computed by oracle_expert_rows_fp8. Routing and
  * the zero-computation experts use the bf16 x unchanged. */
 int64_t oracle_forward_fp8(const uint16_t* x, const uint16_t* wr, const float* bias,
-                           const uint8_t* w13q, const float* w13_scale, const uint16_t* w2,
-                           int64_t T, int64_t d, int64_t N, int64_t Z, int64_t K, int64_t I,
-                           uint16_t* out, float* logits, int32_t* idx, float* gate,
-                           int32_t* counts, double* out_acc) {
+                           const uint8_t* w13q, const float* w13_scale, const uint8_t* w2q,
+                           const float* w2_scale, int64_t T, int64_t d, int64_t N, int64_t Z,
+                           int64_t K, int64_t I, uint16_t* out, float* logits, int32_t* idx,
+                           float* gate, int32_t* counts, double* out_acc) {
     const int64_t E = N + Z;
     oracle_router_logits(x, wr, T, d, E, logits);
     int64_t bad = oracle_route(logits, bias, T, E, K, idx, gate, counts, NULL);
@@ -489,7 +518,8 @@ int64_t oracle_forward_fp8(const uint16_t* x, const uint16_t* wr, const float* b
             const int32_t e = idx[t * K + r];
             const double g = (double)gate[t * K + r];
             if (e < N) {
-                oracle_expert_rows_fp8(xq + t * d, sx + t, &e, 1, d, I, w13q, w13_scale, w2, NULL, yrow);
+                oracle_expert_rows_fp8(xq + t * d, sx + t, &e, 1, d, I, w13q, w13_scale, w2q, w2_scale,
+                                       NULL, yrow);
                 for (int64_t c = 0; c < d; ++c) acc[c] += g * bf16_to_double(yrow[c]);
             } else {
                 for (int64_t c = 0; c < d; ++c) acc[c] += bf16_to_double(x[t * d + c]) * g;  /* E_i(x) = x */

@@ -8,8 +8,10 @@ scale per weight row and per token row, amax / 448) is this library's. What pins
     points (largest finite 448, smallest subnormal 2^-9, saturation, ties to even);
   - row quantisation: the largest element of a row maps to +-448, every element is within half
     a code step of x / s;
-  - the FP8 experts and the FP8 layer reduce exactly to the pinned bf16 oracle when every input
-    is an E4M3 value times a power-of-two scale (then quantisation is exact).
+  - each FP8 projection reduces exactly to the pinned bf16 oracle when its inputs are E4M3
+    values times power-of-two scales (then quantisation is exact): gate/up give the bf16 H bit
+    for bit, the down projection the bf16 Y; the FP8 layer is the MoE-equation combine of its
+    FP8 experts with the bf16 layer's routing.
 """
 import numpy as np
 import pytest
@@ -104,6 +106,8 @@ def exact_fp8_matrix(rng, rows, cols, row_exp):
 
 
 def test_fp8_experts_reduce_to_the_bf16_oracle_on_exact_inputs():
+    """Gate/up operands that quantise exactly give the bf16 oracle's H bit for bit; Y is then the
+    FP8 down projection of that H."""
     rng = np.random.default_rng(9)
     n, d, I, M = 3, 64, 32, 10
     x_codes, xv = exact_fp8_matrix(rng, M, d, rng.integers(-9, -5, M).astype(np.float64))
@@ -115,29 +119,76 @@ def test_fp8_experts_reduce_to_the_bf16_oracle_on_exact_inputs():
     row_expert = rng.integers(0, n, M).astype(np.int32)
     xq, sx = oracle.quantize_rows_e4m3(xb)
     wq, sw = oracle.quantize_rows_e4m3(wb.reshape(n * 2 * I, d))
+    w2q, w2s = oracle.quantize_rows_e4m3(w2.reshape(n * d, I))
     np.testing.assert_array_equal(xq, x_codes)
     np.testing.assert_array_equal(wq, w_codes)
-    h8, y8 = oracle.expert_rows_fp8(xq, sx, row_expert, wq.reshape(n, 2 * I, d), sw.reshape(n, 2 * I), w2)
-    h, y = oracle.expert_rows(xb, row_expert, wb, w2)
+    h8, y8 = oracle.expert_rows_fp8(xq, sx, row_expert, wq.reshape(n, 2 * I, d), sw.reshape(n, 2 * I),
+                                    w2q.reshape(n, d, I), w2s.reshape(n, d))
+    h, _ = oracle.expert_rows(xb, row_expert, wb, w2)
     np.testing.assert_array_equal(h8, h)
-    np.testing.assert_array_equal(y8, y)
+    np.testing.assert_array_equal(y8, oracle.expert_down_fp8(h, row_expert, w2q.reshape(n, d, I), w2s.reshape(n, d)))
 
 
-def test_fp8_layer_reduces_to_the_bf16_layer_on_exact_inputs():
+def test_fp8_down_projection_reduces_to_the_bf16_one_on_exact_inputs():
+    """H rows and W2 rows that quantise exactly: the FP8 down projection is the bf16 one."""
+    rng = np.random.default_rng(12)
+    n, d, I, M = 2, 48, 64, 9
+    _, hv = exact_fp8_matrix(rng, M, I, rng.integers(-6, -2, M).astype(np.float64))
+    _, w2v = exact_fp8_matrix(rng, n * d, I, rng.integers(-16, -12, n * d).astype(np.float64))
+    hb, w2b = bf16_bits(hv), bf16_bits(w2v).reshape(n, d, I)
+    row_expert = rng.integers(0, n, M).astype(np.int32)
+    w2q, w2s = oracle.quantize_rows_e4m3(w2b.reshape(n * d, I))
+    y8 = oracle.expert_down_fp8(hb, row_expert, w2q.reshape(n, d, I), w2s.reshape(n, d))
+    np.testing.assert_array_equal(y8, oracle.expert_down(hb, row_expert, w2b))
+
+
+def test_fp8_down_projection_quantises_each_h_row():
+    """General H rows: Y is the bf16 rounding of the scaled E4M3 product of the row-quantised H
+    and W2 (recomputed here with a float64 matrix product, so allow one bf16 step for a different
+    summation order at a rounding boundary), and differs from the unquantised bf16 Y."""
+    rng = np.random.default_rng(21)
+    n, d, I, M = 2, 40, 128, 16
+    hb = bf16_bits(rng.standard_normal((M, I)) * 0.3)
+    w2b = bf16_bits(rng.standard_normal((n, d, I)) / np.sqrt(I))
+    row_expert = rng.integers(0, n, M).astype(np.int32)
+    w2q, w2s = oracle.quantize_rows_e4m3(w2b.reshape(n * d, I))
+    w2q, w2s = w2q.reshape(n, d, I), w2s.reshape(n, d)
+    y8 = oracle.bf16_bits_to_f64(oracle.expert_down_fp8(hb, row_expert, w2q, w2s))
+    hq, sh = oracle.quantize_rows_e4m3(hb)
+    hdq = oracle.e4m3_to_f64(hq) * sh[:, None].astype(np.float64)
+    wdq = oracle.e4m3_to_f64(w2q) * w2s[:, :, None].astype(np.float64)
+    want = np.stack([wdq[row_expert[r]] @ hdq[r] for r in range(M)])
+    step = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(want), 2.0 ** -126))) - 7)
+    assert np.all(np.abs(y8 - want) <= step)
+    y16 = oracle.bf16_bits_to_f64(oracle.expert_down(hb, row_expert, w2b))
+    assert np.mean(np.abs(y8 - y16) > step) > 0.1
+
+
+def test_fp8_layer_is_the_combine_of_its_fp8_experts():
+    """The FP8 layer routes like the bf16 layer (routing never sees FP8) and its output is the
+    MoE-equation combine of the FP8 experts' rows and the zero-expert identity term."""
     rng = np.random.default_rng(4)
     T, d, N, Z, K, I = 12, 64, 4, 2, 3, 32
-    _, xv = exact_fp8_matrix(rng, T, d, rng.integers(-8, -5, T).astype(np.float64))
-    _, wv = exact_fp8_matrix(rng, N * 2 * I, d, rng.integers(-13, -10, N * 2 * I).astype(np.float64))
-    xb, w13 = bf16_bits(xv), bf16_bits(wv).reshape(N, 2 * I, d)
+    xb = bf16_bits(rng.standard_normal((T, d)))
+    w13 = bf16_bits(rng.standard_normal((N, 2 * I, d)) / np.sqrt(d))
+    w2 = bf16_bits(rng.standard_normal((N, d, I)) / np.sqrt(I))
     wr = bf16_bits(rng.integers(-4, 5, (N + Z, d)) * 2.0 ** -6)
-    w2 = bf16_bits(rng.standard_normal((N, d, I)) * 0.05)
     bias = np.zeros(N + Z, np.float32)
     wq, sw = oracle.quantize_rows_e4m3(w13.reshape(N * 2 * I, d))
-    f8 = oracle.forward_fp8(xb, wr, bias, wq.reshape(N, 2 * I, d), sw.reshape(N, 2 * I), w2, N, Z, K)
+    w2q, w2s = oracle.quantize_rows_e4m3(w2.reshape(N * d, I))
+    wq, sw, w2q, w2s = wq.reshape(N, 2 * I, d), sw.reshape(N, 2 * I), w2q.reshape(N, d, I), w2s.reshape(N, d)
+    f8 = oracle.forward_fp8(xb, wr, bias, wq, sw, w2q, w2s, N, Z, K)
     ref = oracle.forward(xb, wr, bias, w13, w2, N, Z, K)
-    for k in ("idx", "gate", "counts", "logits", "out"):
+    for k in ("idx", "gate", "counts", "logits"):
         np.testing.assert_array_equal(f8[k], ref[k], err_msg=k)
-    np.testing.assert_array_equal(f8["out_exact"], ref["out_exact"])
+    offsets, row_token, pair_row = oracle.permute(f8["idx"], N)
+    row_expert = np.repeat(np.arange(N, dtype=np.int32), np.diff(offsets))
+    xq, sx = oracle.quantize_rows_e4m3(xb)
+    _, y = oracle.expert_rows_fp8(np.ascontiguousarray(xq[row_token]), np.ascontiguousarray(sx[row_token]),
+                                  row_expert, wq, sw, w2q, w2s, want_h=False)
+    out, exact = oracle.combine(xb, y, f8["idx"], f8["gate"], pair_row, N, want_exact=True)
+    np.testing.assert_array_equal(f8["out"], out)
+    np.testing.assert_array_equal(f8["out_exact"], exact)
 
 
 def test_fp8_layer_on_general_inputs_is_close_to_but_not_the_bf16_layer():
@@ -149,7 +200,9 @@ def test_fp8_layer_on_general_inputs_is_close_to_but_not_the_bf16_layer():
     wr = bf16_bits(rng.integers(-4, 5, (N + Z, d)) * 2.0 ** -6)
     bias = np.zeros(N + Z, np.float32)
     wq, sw = oracle.quantize_rows_e4m3(w13.reshape(N * 2 * I, d))
-    f8 = oracle.forward_fp8(xb, wr, bias, wq.reshape(N, 2 * I, d), sw.reshape(N, 2 * I), w2, N, Z, K)
+    w2q, w2s = oracle.quantize_rows_e4m3(w2.reshape(N * d, I))
+    f8 = oracle.forward_fp8(xb, wr, bias, wq.reshape(N, 2 * I, d), sw.reshape(N, 2 * I),
+                            w2q.reshape(N, d, I), w2s.reshape(N, d), N, Z, K)
     ref = oracle.forward(xb, wr, bias, w13, w2, N, Z, K)
     np.testing.assert_array_equal(f8["idx"], ref["idx"])          # routing does not see FP8
     diff = np.abs(f8["out_exact"] - ref["out_exact"])

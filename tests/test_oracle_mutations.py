@@ -81,6 +81,14 @@ MUTATIONS = [
      "U += xd[k] * ((double)su[j] * oracle_e4m3_to_double(wu[j * d + k]));",
      "U += xd[k] * ((double)sg[j] * oracle_e4m3_to_double(wu[j * d + k]));",
      fp8pins.test_fp8_experts_reduce_to_the_bf16_oracle_on_exact_inputs),
+    ("FP8: down projection scaled by the wrong weight row",
+     "acc += hd[j] * ((double)w2s[i] * oracle_e4m3_to_double(w2q[i * I + j]));",
+     "acc += hd[j] * ((double)w2s[(i + 1) % d] * oracle_e4m3_to_double(w2q[i * I + j]));",
+     fp8pins.test_fp8_down_projection_reduces_to_the_bf16_one_on_exact_inputs),
+    ("FP8: H not quantised before the down projection",
+     "for (int64_t j = 0; j < I; ++j) hd[j] = (double)sh * oracle_e4m3_to_double(hq[j]);",
+     "for (int64_t j = 0; j < I; ++j) hd[j] = bf16_to_double(hrow[j]) * (sh > 0.0f ? 1.0 : 1.0);",
+     fp8pins.test_fp8_down_projection_quantises_each_h_row),
     ("FP8: E4M3 exponent bias 8 instead of 7",
      "ldexp(1.0 + m / 8.0, e - 7);",
      "ldexp(1.0 + m / 8.0, e - 8);",
