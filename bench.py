@@ -166,6 +166,7 @@ def run_ours(args):
     if f8:
         # weights are quantised once, outside the timed region (an offline step for a deployment)
         w13q, w13s = B.lc_moe_quantize_e4m3(w13)
+        w2q, w2s = B.lc_moe_quantize_e4m3(w2)
         torch.cuda.synchronize(dev)
     ws = B.new_workspace(shape, B.OP_FORWARD_FP8 if f8 else B.OP_FORWARD, dev)
     out = torch.empty(T, w.d, dtype=torch.bfloat16, device=dev)
@@ -175,7 +176,7 @@ def run_ours(args):
 
     def forward(xin, o, events=None):
         if f8:
-            B.lc_moe_forward_fp8(xin, wr, bias, w13q, w13s, w2, K, out=o, counts=counts, ws=ws,
+            B.lc_moe_forward_fp8(xin, wr, bias, w13q, w13s, w2q, w2s, K, out=o, counts=counts, ws=ws,
                                  stream=stream, events=events)
         else:
             B.lc_moe_forward(xin, wr, bias, w13, w2, K, out=o, counts=counts, ws=ws, stream=stream,
@@ -291,8 +292,8 @@ def run_ours(args):
     # ---- roofline of each stage (algorithmic work only)
     peaks, peak_src = load_peaks()
     d_, I_ = w.d, w.I
-    # E4M3 gate/up weights take 1 byte per element; the down projection stays bf16
-    wbytes_touched = touched * d_ * I_ * ((2 + 2) if f8 else 6)
+    # E4M3 expert weights take 1 byte per element
+    wbytes_touched = touched * d_ * I_ * (3 if f8 else 6)
     # tensor peak of each contraction: bf16 measured; E4M3 = 2 x bf16 (nominal dense ratio 4.5/2.25)
     peak16 = peaks["bf16_tflops_sustained"]
     peak_g1 = 2.0 * peak16 if f8 else peak16
@@ -314,7 +315,7 @@ def run_ours(args):
         t_s = mean[j] / 1e3
         if bound == "tensor":
             ach = work / t_s / 1e12
-            peak = peak_g1 if name == "gemm1_swiglu" else peaks["bf16_tflops_sustained"]
+            peak = peak_g1 if name in ("gemm1_swiglu", "gemm2_down") else peaks["bf16_tflops_sustained"]
             unit = "TFLOP/s"
         else:
             ach = work / t_s / 1e9
@@ -331,7 +332,7 @@ def run_ours(args):
                 "unit": ds["unit"], "frac": ds["frac"],
                 "peak_source": (f"{peak_src} ("
                                 + ("2 x bf16_tflops_sustained, the nominal E4M3/bf16 dense ratio"
-                                   if f8 and dom == "gemm1_swiglu" else
+                                   if f8 and dom in ("gemm1_swiglu", "gemm2_down") else
                                    "bf16_tflops_sustained" if ds["bound"] == "tensor" else "hbm_gbs")
                                 + ", MEASURED_PEAKS.json)") if peak_src == "measured" else "fallback",
                 "traffic": (trec["dram_bytes_per_launch"] if trec else None),
@@ -339,21 +340,21 @@ def run_ours(args):
     # whole-step roofline: max(FLOP / sustained TC peak, touched weights + activations / HBM)
     flops = 2.0 * T * d_ * E + 6.0 * M * d_ * I_
     bytes_ = wbytes_touched + E * d_ * 2 + 2 * T * d_ * 2
-    t_tc = (2.0 * T * d_ * E + 2.0 * M * d_ * I_) / (peak16 * 1e12) + 4.0 * M * d_ * I_ / (peak_g1 * 1e12)
+    t_tc = 2.0 * T * d_ * E / (peak16 * 1e12) + 6.0 * M * d_ * I_ / (peak_g1 * 1e12)
     t_roof = max(t_tc, bytes_ / (peaks["hbm_gbs"] * 1e9))
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3 gate/up + bf16" if f8 else "bf16",
+        "dtype": "e4m3 experts + bf16 router/combine" if f8 else "bf16",
         "data": "synthetic (seeded; random-init weights of the LongCat-Flash MoE-layer shape)",
         "config": {"workload": f"{w.name}: MoE layer with zero-computation experts, T={T} tokens per GPU",
                    "T": T, "d": d_, "N": w.N, "Z": w.Z, "K": K, "K_e": w.K_e, "I": I_,
                    "router": w.router, "mu": w.mu, "parallelism": f"dp{world}",
                    "step": "forward + counts all-reduce (N>1) + expert-bias update",
-                   "experts": ("gate/up projections on E4M3 codes with one fp32 scale per weight row "
-                               "and per token row (weights quantised once before timing), down "
-                               "projection bf16") if f8 else "bf16",
+                   "experts": ("all expert projections on E4M3 codes with one fp32 scale per weight "
+                               "row and per activation row (weights quantised once before timing)")
+                              if f8 else "bf16",
                    "l2": f"inputs larger than L2 ({w.weight_bytes() / 1e9:.1f} GB expert weights, "
                          f"{T * d_ * 2 / 1e6:.0f} MB x per step)"},
         "roofline": roofline,
@@ -370,10 +371,10 @@ def run_ours(args):
                 "d2h_bytes_per_step": int(out.numel() * 2), "steps": e2e_steps_n,
                 "copies": "pinned host x -> device and out -> pinned host every step, on a copy "
                           "stream overlapping the neighbouring steps' compute"},
-        "gpu_launches": int(args.steps * (sum(KERNELS_PER_STAGE) + 1 + (1 if f8 else 0))),
+        "gpu_launches": int(args.steps * (sum(KERNELS_PER_STAGE) + 1 + (2 if f8 else 0))),
         "gpu_launches_note": "kernels of this library inside the device-timed region: "
-                             f"{sum(KERNELS_PER_STAGE) + (1 if f8 else 0)} per forward "
-                             f"{'(incl. the token-row quantiser) ' if f8 else ''}+ 1 bias update, per step",
+                             f"{sum(KERNELS_PER_STAGE) + (2 if f8 else 0)} per forward "
+                             f"{'(incl. the token-row and H-row quantisers) ' if f8 else ''}+ 1 bias update, per step",
         "clocks": ClockSampler.summarize(clock_rows),
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline and not f8:
@@ -583,7 +584,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time")
     ap.add_argument("--ref-tokens", type=int, default=4, help="tokens per reference-arm step")
     ap.add_argument("--experts", choices=["bf16", "fp8"], default="bf16",
-                    help="fp8: E4M3 gate/up projections (lc_moe_forward_fp8)")
+                    help="fp8: E4M3 expert projections (lc_moe_forward_fp8)")
     ap.add_argument("--sweep", choices=["ffn_rows", "hist"], default=None,
                     help="run a kernel sweep instead of the step (one GPU)")
     args = ap.parse_args()

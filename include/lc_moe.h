@@ -79,7 +79,7 @@ enum {
     LC_MOE_OP_ROUTE = 1,     /* lc_moe_route */
     LC_MOE_OP_PERMUTE = 2,   /* lc_moe_permute */
     LC_MOE_OP_STATUS = 3,    /* every other entry point: the status word only (256 bytes) */
-    LC_MOE_OP_FORWARD_FP8 = 4  /* lc_moe_forward_fp8 / lc_moe_forward_fp8_timed (0 if d % 128) */
+    LC_MOE_OP_FORWARD_FP8 = 4  /* lc_moe_forward_fp8 / _timed (0 unless d and I are multiples of 128) */
 };
 
 /* Stages of lc_moe_forward, in launch order (lc_moe_forward_timed records one event before
@@ -226,9 +226,11 @@ int lc_moe_permute_noalloc(const lc_moe_shape* s, const int32_t* idx, const void
  * Section 5 of the LongCat-Flash llm-wiki entity page (inference and deployment) lists FP8/BF16
  * quantisation and an FP8 deployment on one node, without a scaling scheme. This library's
  * scheme: E4M3 codes (OCP 8-bit floating point: 4 exponent bits, bias 7, 3 mantissa bits, largest
- * finite 448) with one fp32 scale per row, s = amax / 448, x ~ s * code. The gate and up
- * projections run on E4M3 tensor-core operands (tcgen05 kind::f8f6f4, fp32 accumulation); the
- * down projection, routing, combine and the zero-computation experts stay as in lc_moe_forward.
+ * finite 448) with one fp32 scale per row, s = amax / 448, x ~ s * code. All three expert
+ * projections run on E4M3 tensor-core operands (tcgen05 kind::f8f6f4, fp32 accumulation): the
+ * activation rows (token rows of x, rows of H after their bf16 rounding) are quantised per row
+ * on the device, the weights once by the caller. Routing, the combine and the zero-computation
+ * experts stay as in lc_moe_forward.
  */
 
 /* Row-wise E4M3 quantisation of a bf16 matrix src [rows, cols] (cols a multiple of 8):
@@ -239,24 +241,28 @@ int lc_moe_permute_noalloc(const lc_moe_shape* s, const int32_t* idx, const void
 int lc_moe_quantize_e4m3(const void* src, int64_t rows, int32_t cols, void* dst, float* scale,
                          void* stream);
 
-/* lc_moe_forward with E4M3 gate/up projections:
- *   w13q      [N, 2I, d] E4M3 codes of W13 (as lc_moe_quantize_e4m3 makes them)
+/* lc_moe_forward with E4M3 experts:
+ *   w13q      [N, 2I, d] E4M3 codes of W13 (as lc_moe_quantize_e4m3 makes them from [N*2I, d])
  *   w13_scale [N, 2I]    fp32 scale of each W13 row (16-byte aligned)
- * Each token row x_t is quantised the same way (one scale per token) before the gate/up GEMM;
- * G = (sum_k code_x code_g) * s_x * s_g and U likewise, in fp32, then the SwiGLU and the rest
- * of the layer as lc_moe_forward. Needs d % 128 == 0 (else LC_MOE_ERR_UNSUPPORTED_SHAPE).
- * ws: lc_moe_workspace_bytes(s, LC_MOE_OP_FORWARD_FP8) bytes. */
+ *   w2q       [N, d, I]  E4M3 codes of W2 (from [N*d, I])
+ *   w2_scale  [N, d]     fp32 scale of each W2 row (16-byte aligned)
+ * Each token row x_t is quantised the same way (one scale per token) before the gate/up GEMM:
+ * G = (sum_k code_x code_g) * s_x * s_g and U likewise, in fp32; H = bf16(silu(G) * U); each H
+ * row is quantised (one scale per row) and Y = bf16((sum_j code_h code_w) * s_h * s_w). The
+ * rest of the layer is lc_moe_forward's. Needs d and I multiples of 128 (else
+ * LC_MOE_ERR_UNSUPPORTED_SHAPE). ws: lc_moe_workspace_bytes(s, LC_MOE_OP_FORWARD_FP8) bytes. */
 int lc_moe_forward_fp8(const lc_moe_shape* s, const void* x, const void* wr, const float* bias,
-                       const void* w13q, const float* w13_scale, const void* w2, void* out,
-                       int32_t* idx, float* gate, int32_t* counts, void* ws, size_t ws_bytes,
-                       void* stream);
+                       const void* w13q, const float* w13_scale, const void* w2q,
+                       const float* w2_scale, void* out, int32_t* idx, float* gate, int32_t* counts,
+                       void* ws, size_t ws_bytes, void* stream);
 
 /* lc_moe_forward_fp8 plus the stage events of lc_moe_forward_timed (the gather stage also holds
- * the quantisation of the token rows). */
+ * the quantisation of the token rows, the GEMM 2 stage that of the H rows). */
 int lc_moe_forward_fp8_timed(const lc_moe_shape* s, const void* x, const void* wr, const float* bias,
-                             const void* w13q, const float* w13_scale, const void* w2, void* out,
-                             int32_t* idx, float* gate, int32_t* counts, void* ws, size_t ws_bytes,
-                             void* stream, void* const* events);
+                             const void* w13q, const float* w13_scale, const void* w2q,
+                             const float* w2_scale, void* out, int32_t* idx, float* gate,
+                             int32_t* counts, void* ws, size_t ws_bytes, void* stream,
+                             void* const* events);
 
 #ifdef __cplusplus
 }

@@ -86,7 +86,7 @@ def _configure(L: ctypes.CDLL) -> ctypes.CDLL:
     L.lc_moe_combine.argtypes = [SP, P, P, P, P, P, P, SZ, P]
     L.lc_moe_permute_noalloc.argtypes = [SP, P, P, P, P, P, P, P, P]
     L.lc_moe_quantize_e4m3.argtypes = [P, I64, I32, P, P, P]
-    fwd8 = [SP, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+    fwd8 = [SP, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
     L.lc_moe_forward_fp8.argtypes = fwd8
     L.lc_moe_forward_fp8_timed.argtypes = fwd8 + [ctypes.POINTER(P)]
     return L
@@ -215,10 +215,11 @@ def lc_moe_quantize_e4m3(src, dst=None, scale=None, stream=None):
     return dst, scale
 
 
-def lc_moe_forward_fp8(x, wr, bias, w13q, w13_scale, w2, K: int, out=None, idx=None, gate=None,
-                       counts=None, ws=None, stream=None, events=None):
-    """MoE(x) with E4M3 gate/up projections: w13q [N, 2I, d] uint8 codes and w13_scale [N, 2I]
-    float32 (from lc_moe_quantize_e4m3); w2 [N, d, I] bf16. Returns ``out`` [T, d] bf16."""
+def lc_moe_forward_fp8(x, wr, bias, w13q, w13_scale, w2q, w2_scale, K: int, out=None, idx=None,
+                       gate=None, counts=None, ws=None, stream=None, events=None):
+    """MoE(x) with E4M3 experts: w13q [N, 2I, d] / w2q [N, d, I] uint8 codes with row scales
+    w13_scale [N, 2I] / w2_scale [N, d] float32 (from lc_moe_quantize_e4m3). Returns ``out``
+    [T, d] bf16."""
     T, d = x.shape
     E = wr.shape[0]
     N, two_i, _ = w13q.shape
@@ -228,7 +229,8 @@ def lc_moe_forward_fp8(x, wr, bias, w13q, w13_scale, w2, K: int, out=None, idx=N
     _need(bias, torch.float32, (E,), "bias")
     _need(w13q, torch.uint8, (N, 2 * I, d), "w13q")
     _need(w13_scale, torch.float32, (N, 2 * I), "w13_scale")
-    _need(w2, torch.bfloat16, (N, d, I), "w2")
+    _need(w2q, torch.uint8, (N, d, I), "w2q")
+    _need(w2_scale, torch.float32, (N, d), "w2_scale")
     if out is None:
         out = torch.empty(T, d, dtype=torch.bfloat16, device=x.device)
     _need(out, torch.bfloat16, (T, d), "out")
@@ -241,8 +243,9 @@ def lc_moe_forward_fp8(x, wr, bias, w13q, w13_scale, w2, K: int, out=None, idx=N
     s = Shape(T, d, N, E - N, K, I)
     if ws is None:
         ws = new_workspace(s, OP_FORWARD_FP8, x.device)
-    args = [ctypes.byref(s), _ptr(x), _ptr(wr), _ptr(bias), _ptr(w13q), _ptr(w13_scale), _ptr(w2),
-            _ptr(out), _ptr(idx), _ptr(gate), _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)]
+    args = [ctypes.byref(s), _ptr(x), _ptr(wr), _ptr(bias), _ptr(w13q), _ptr(w13_scale), _ptr(w2q),
+            _ptr(w2_scale), _ptr(out), _ptr(idx), _ptr(gate), _ptr(counts), _ptr(ws), ws.numel(),
+            _stream(stream)]
     if events is None:
         _check(_lib().lc_moe_forward_fp8(*args), "lc_moe_forward_fp8")
     else:

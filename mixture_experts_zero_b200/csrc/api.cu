@@ -37,12 +37,14 @@ int check_shape(const lc_moe_shape* s) {
 
 // Byte offsets of the forward workspace regions.
 struct FwdLayout {
-    size_t logits, idx, gate, offsets, row_token, pair_row, scratch, xq, sx, s_row, x_perm, h, y, total;
+    size_t logits, idx, gate, offsets, row_token, pair_row, scratch, xq, sx, s_row, x_perm, h, hq, s_h, y,
+        total;
     int64_t rows_cap;
 };
 
 // f8: the E4M3 variant (quantised token rows [T, d] bytes and their scales [T], grouped rows of
-// d bytes with their scales [rows_cap]); otherwise grouped rows of d bf16 values.
+// d bytes with their scales [rows_cap], quantised H rows [rows_cap, I] bytes with their scales);
+// otherwise grouped rows of d bf16 values.
 FwdLayout fwd_layout(const lc_moe_shape* s, bool f8 = false) {
     FwdLayout L{};
     const size_t T = s->T, K = s->K, E = static_cast<size_t>(s->N) + s->Z;
@@ -62,6 +64,10 @@ FwdLayout fwd_layout(const lc_moe_shape* s, bool f8 = false) {
     }
     L.x_perm = o;    o = align_up(o + static_cast<size_t>(rows_cap) * s->d * (f8 ? 1 : 2));
     L.h = o;         o = align_up(o + static_cast<size_t>(rows_cap) * s->I * 2);
+    if (f8) {
+        L.hq = o;    o = align_up(o + static_cast<size_t>(rows_cap) * s->I);
+        L.s_h = o;   o = align_up(o + static_cast<size_t>(rows_cap) * 4);
+    }
     L.y = o;         o = align_up(o + static_cast<size_t>(rows_cap) * s->d * 2);
     L.total = o;
     L.rows_cap = rows_cap;
@@ -104,18 +110,18 @@ int record(void* const* events, int i, cudaStream_t st) {
 }
 
 int forward_impl(const lc_moe_shape* s, const void* x, const void* wr, const float* bias,
-                 const void* w13, const float* w13_scale, const void* w2, void* out, int32_t* idx,
-                 float* gate, int32_t* counts, void* ws, size_t ws_bytes, void* stream,
-                 void* const* events) {
-    // w13_scale != NULL selects the E4M3 experts (w13 then holds E4M3 codes)
+                 const void* w13, const float* w13_scale, const void* w2, const float* w2_scale,
+                 void* out, int32_t* idx, float* gate, int32_t* counts, void* ws, size_t ws_bytes,
+                 void* stream, void* const* events) {
+    // w13_scale != NULL selects the E4M3 experts (w13 and w2 then hold E4M3 codes)
     const bool f8 = w13_scale != nullptr;
     LC_TRY(check_shape(s));
-    if (f8 && s->d % 128) return LC_MOE_ERR_UNSUPPORTED_SHAPE;
-    if (!x || !wr || !bias || !w13 || !w2 || !out || !ws) return LC_MOE_ERR_INVALID_ARG;
+    if (f8 && (s->d % 128 || s->I % 128)) return LC_MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!x || !wr || !bias || !w13 || !w2 || !out || !ws || (f8 && !w2_scale)) return LC_MOE_ERR_INVALID_ARG;
     const FwdLayout L = fwd_layout(s, f8);
     if (ws_bytes < L.total) return LC_MOE_ERR_WORKSPACE_TOO_SMALL;
     for (const void* p : {x, wr, static_cast<const void*>(bias), w13, static_cast<const void*>(w13_scale), w2,
-                          static_cast<const void*>(out),
+                          static_cast<const void*>(w2_scale), static_cast<const void*>(out),
                           static_cast<const void*>(idx), static_cast<const void*>(gate),
                           static_cast<const void*>(counts), static_cast<const void*>(ws)})
         if (p && !aligned16(p)) return LC_MOE_ERR_MISALIGNED;
@@ -158,7 +164,16 @@ int forward_impl(const lc_moe_shape* s, const void* x, const void* wr, const flo
         LC_CUDA(launch_grouped_swiglu(x_perm, L.rows_cap, offsets, s->N, w13, s->d, s->I, h, status, st));
     }
     LC_TRY(record(events, LC_MOE_STAGE_GEMM2, st));
-    LC_CUDA(launch_grouped_down(h, L.rows_cap, offsets, s->N, w2, s->d, s->I, y, status, st));
+    if (f8) {
+        // quantise the offsets[N] rows of H that GEMM 1 wrote, one scale per row
+        void* hq = at<void>(ws, L.hq);
+        float* s_h = at<float>(ws, L.s_h);
+        LC_CUDA(launch_quantize_rows_e4m3(h, L.rows_cap, s->I, hq, s_h, st, offsets + s->N));
+        LC_CUDA(launch_grouped_down_e4m3(hq, s_h, L.rows_cap, offsets, s->N, w2, w2_scale, s->d, s->I, y,
+                                         status, st));
+    } else {
+        LC_CUDA(launch_grouped_down(h, L.rows_cap, offsets, s->N, w2, s->d, s->I, y, status, st));
+    }
     LC_TRY(record(events, LC_MOE_STAGE_COMBINE, st));
     LC_CUDA(launch_combine(x, y, gate_w, pair_row, s->T, s->d, s->K, out, st));
     LC_TRY(record(events, LC_MOE_NUM_STAGES, st));
@@ -216,7 +231,7 @@ size_t lc_moe_workspace_bytes(const lc_moe_shape* s, int op) {
     if (check_shape(s) != LC_MOE_OK) return 0;
     switch (op) {
         case LC_MOE_OP_FORWARD: return fwd_layout(s).total;
-        case LC_MOE_OP_FORWARD_FP8: return s->d % 128 ? 0 : fwd_layout(s, true).total;
+        case LC_MOE_OP_FORWARD_FP8: return (s->d % 128 || s->I % 128) ? 0 : fwd_layout(s, true).total;
         case LC_MOE_OP_ROUTE: return route_ws_bytes(s);
         case LC_MOE_OP_PERMUTE: return permute_ws_bytes(s);
         case LC_MOE_OP_STATUS: return kStatusBytes;
@@ -232,7 +247,7 @@ void lc_moe_set_wait_limit_ns(uint64_t limit_ns) {
 int lc_moe_forward(const lc_moe_shape* s, const void* x, const void* wr, const float* bias,
                    const void* w13, const void* w2, void* out, int32_t* idx, float* gate,
                    int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
-    return forward_impl(s, x, wr, bias, w13, nullptr, w2, out, idx, gate, counts, ws, ws_bytes, stream,
+    return forward_impl(s, x, wr, bias, w13, nullptr, w2, nullptr, out, idx, gate, counts, ws, ws_bytes, stream,
                         nullptr);
 }
 
@@ -243,28 +258,29 @@ int lc_moe_forward_timed(const lc_moe_shape* s, const void* x, const void* wr, c
     if (!events) return LC_MOE_ERR_INVALID_ARG;
     for (int i = 0; i <= LC_MOE_NUM_STAGES; ++i)
         if (!events[i]) return LC_MOE_ERR_INVALID_ARG;
-    return forward_impl(s, x, wr, bias, w13, nullptr, w2, out, idx, gate, counts, ws, ws_bytes, stream,
+    return forward_impl(s, x, wr, bias, w13, nullptr, w2, nullptr, out, idx, gate, counts, ws, ws_bytes, stream,
                         events);
 }
 
 int lc_moe_forward_fp8(const lc_moe_shape* s, const void* x, const void* wr, const float* bias,
-                       const void* w13q, const float* w13_scale, const void* w2, void* out,
-                       int32_t* idx, float* gate, int32_t* counts, void* ws, size_t ws_bytes,
-                       void* stream) {
-    if (!w13_scale) return LC_MOE_ERR_INVALID_ARG;
-    return forward_impl(s, x, wr, bias, w13q, w13_scale, w2, out, idx, gate, counts, ws, ws_bytes,
-                        stream, nullptr);
+                       const void* w13q, const float* w13_scale, const void* w2q,
+                       const float* w2_scale, void* out, int32_t* idx, float* gate, int32_t* counts,
+                       void* ws, size_t ws_bytes, void* stream) {
+    if (!w13_scale || !w2_scale) return LC_MOE_ERR_INVALID_ARG;
+    return forward_impl(s, x, wr, bias, w13q, w13_scale, w2q, w2_scale, out, idx, gate, counts, ws,
+                        ws_bytes, stream, nullptr);
 }
 
 int lc_moe_forward_fp8_timed(const lc_moe_shape* s, const void* x, const void* wr, const float* bias,
-                             const void* w13q, const float* w13_scale, const void* w2, void* out,
-                             int32_t* idx, float* gate, int32_t* counts, void* ws, size_t ws_bytes,
-                             void* stream, void* const* events) {
-    if (!w13_scale || !events) return LC_MOE_ERR_INVALID_ARG;
+                             const void* w13q, const float* w13_scale, const void* w2q,
+                             const float* w2_scale, void* out, int32_t* idx, float* gate,
+                             int32_t* counts, void* ws, size_t ws_bytes, void* stream,
+                             void* const* events) {
+    if (!w13_scale || !w2_scale || !events) return LC_MOE_ERR_INVALID_ARG;
     for (int i = 0; i <= LC_MOE_NUM_STAGES; ++i)
         if (!events[i]) return LC_MOE_ERR_INVALID_ARG;
-    return forward_impl(s, x, wr, bias, w13q, w13_scale, w2, out, idx, gate, counts, ws, ws_bytes,
-                        stream, events);
+    return forward_impl(s, x, wr, bias, w13q, w13_scale, w2q, w2_scale, out, idx, gate, counts, ws,
+                        ws_bytes, stream, events);
 }
 
 int lc_moe_quantize_e4m3(const void* src, int64_t rows, int32_t cols, void* dst, float* scale,

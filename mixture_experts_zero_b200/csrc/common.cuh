@@ -348,12 +348,20 @@ cudaError_t launch_gather_e4m3(const void* xq, const float* sx, int T, int d, in
 
 // Row-wise E4M3 quantisation of a bf16 matrix [R, C] (C % 8 == 0): scale[r] = amax / 448
 // (1 for an all-zero row), dst[r, c] = E4M3(src[r, c] / scale[r]) (round to nearest even,
-// saturating at 448).
+// saturating at 448). With rows_dev, only the first min(R, *rows_dev) rows (a count on the
+// device, e.g. offsets[N]) are quantised.
 cudaError_t launch_quantize_rows_e4m3(const void* src, int64_t R, int C, void* dst, float* scale,
-                                      cudaStream_t st);
+                                      cudaStream_t st, const int32_t* rows_dev = nullptr);
 
 // Grouped GEMM 1 on E4M3 operands: rows x_perm [rows_cap, d] (codes) with row scales s_row,
 // W13 codes [N, 2I, d] with one scale per weight row; the SwiGLU epilogue applies both scales.
+// Grouped GEMM 2 on E4M3 operands: hq [rows_cap, I] codes with row scales s_h, W2 codes
+// [N, d, I] with one scale per weight row (output feature).
+cudaError_t launch_grouped_down_e4m3(const void* hq, const float* s_h, int64_t rows_cap,
+                                     const int32_t* offsets, int N, const void* w2q,
+                                     const float* w2_scale, int d, int I, void* y, uint32_t* status,
+                                     cudaStream_t st);
+
 cudaError_t launch_grouped_swiglu_e4m3(const void* x_perm, const float* s_row, int64_t rows_cap,
                                        const int32_t* offsets, int N, const void* w13q,
                                        const float* w13_scale, int d, int I, void* h,

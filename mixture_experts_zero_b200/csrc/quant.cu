@@ -24,8 +24,12 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
 
 __global__ void __launch_bounds__(QUANT_THREADS)
     quantize_rows_kernel(const uint4* __restrict__ src, int64_t R, int c8, uint2* __restrict__ dst,
-                         float* __restrict__ scale) {
+                         float* __restrict__ scale, const int32_t* __restrict__ rows_dev) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (rows_dev) {
+        const int64_t rd = *rows_dev;
+        if (rd < R) R = rd < 0 ? 0 : rd;
+    }
     const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (QUANT_THREADS / 32);
     for (int64_t r = static_cast<int64_t>(blockIdx.x) * (QUANT_THREADS / 32) + warp; r < R;
          r += warps_total) {
@@ -59,7 +63,7 @@ __global__ void __launch_bounds__(QUANT_THREADS)
 }  // namespace
 
 cudaError_t launch_quantize_rows_e4m3(const void* src, int64_t R, int C, void* dst, float* scale,
-                                      cudaStream_t st) {
+                                      cudaStream_t st, const int32_t* rows_dev) {
     const DevInfo* di = current_device_info();
     if (!di) return cudaErrorUnknown;
     if (R == 0) return cudaSuccess;
@@ -67,7 +71,7 @@ cudaError_t launch_quantize_rows_e4m3(const void* src, int64_t R, int C, void* d
     int64_t blocks = (R + warps - 1) / warps;
     if (blocks > static_cast<int64_t>(di->sm_count) * 16) blocks = static_cast<int64_t>(di->sm_count) * 16;
     quantize_rows_kernel<<<static_cast<int>(blocks), QUANT_THREADS, 0, st>>>(
-        static_cast<const uint4*>(src), R, C / 8, static_cast<uint2*>(dst), scale);
+        static_cast<const uint4*>(src), R, C / 8, static_cast<uint2*>(dst), scale, rows_dev);
     return cudaGetLastError();
 }
 

@@ -450,6 +450,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         tmem_ld_wait();
                         const int f0 = tl.n0 + c;
                         if (valid && f0 < g.n_out) {
+                            if (F8) {
+                                // (acc * row scale) * weight-row scale
+                                const float sr = __ldg(g.row_scale + grow);
+                                const float4* sw4 = reinterpret_cast<const float4*>(
+                                    g.w_scale + static_cast<int64_t>(tl.grp) * g.b_group_rows + f0);
+#pragma unroll
+                                for (int j4 = 0; j4 < 8; ++j4) {
+                                    const float4 a = __ldg(sw4 + j4);
+                                    const float sa[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                                    for (int u = 0; u < 4; ++u)
+                                        v[4 * j4 + u] = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j4 + u]), sr), sa[u]));
+                                }
+                            }
                             uint32_t pk[16];
 #pragma unroll
                             for (int j = 0; j < 16; ++j)
@@ -494,6 +508,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                             v[j] = __float_as_uint(silu_mul(__uint_as_float(v[j]), __uint_as_float(uv[j])));
                     } else {
                         tmem_ld_wait();
+                        if (F8) {
+                            const int fl = f0 + lane < g.n_out ? f0 + lane : g.n_out - 1;
+                            const float sw = __ldg(g.w_scale + static_cast<int64_t>(tl.grp) * g.b_group_rows + fl);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                int64_t rr = tl.row0 + c0 + j;
+                                if (rr >= g.rows_cap) rr = g.rows_cap - 1;
+                                v[j] = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(v[j]), __ldg(g.row_scale + rr)), sw));
+                            }
+                        }
                     }
                     // lane = feature f0 + lane, v[j] = value for row c0 + j
 #pragma unroll
@@ -611,15 +635,10 @@ cudaError_t launch_grouped_swiglu_e4m3(const void* x_perm, const float* s_row, i
     return launch_pair<MODE_SWIGLU, true>(mr, mw, mt, a, pair_grid(di), st);
 }
 
-cudaError_t launch_grouped_down(const void* h, int64_t rows_cap, const int32_t* offsets, int N,
-                                const void* w2, int d, int I, void* y, uint32_t* status,
-                                cudaStream_t st) {
-    const DevInfo* di = current_device_info();
-    if (!di) return cudaErrorUnknown;
-    CUtensorMap mr, mw, mt;
-    if (!make_tma_map_2d(&mr, h, static_cast<uint64_t>(rows_cap), I, HALF_M)) return cudaErrorInvalidValue;
-    if (!make_tma_map_2d(&mw, w2, static_cast<uint64_t>(N) * d, I, HALF_M)) return cudaErrorInvalidValue;
-    if (!make_tma_map_2d(&mt, h, static_cast<uint64_t>(rows_cap), I, TOK_BOX)) return cudaErrorInvalidValue;
+namespace {
+
+PairArgs down_args(int64_t rows_cap, const int32_t* offsets, int N, int d, int I, void* y,
+                   uint32_t* status) {
     PairArgs a{};
     a.offsets = offsets;
     a.out = static_cast<__nv_bfloat16*>(y);
@@ -637,7 +656,38 @@ cudaError_t launch_grouped_down(const void* h, int64_t rows_cap, const int32_t* 
     a.s_tiles = (d + 2 * HALF_M - 1) / (2 * HALF_M);
     a.cold_rows = 256;
     a.rem_rows = 256;
+    return a;
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_down(const void* h, int64_t rows_cap, const int32_t* offsets, int N,
+                                const void* w2, int d, int I, void* y, uint32_t* status,
+                                cudaStream_t st) {
+    const DevInfo* di = current_device_info();
+    if (!di) return cudaErrorUnknown;
+    CUtensorMap mr, mw, mt;
+    if (!make_tma_map_2d(&mr, h, static_cast<uint64_t>(rows_cap), I, HALF_M)) return cudaErrorInvalidValue;
+    if (!make_tma_map_2d(&mw, w2, static_cast<uint64_t>(N) * d, I, HALF_M)) return cudaErrorInvalidValue;
+    if (!make_tma_map_2d(&mt, h, static_cast<uint64_t>(rows_cap), I, TOK_BOX)) return cudaErrorInvalidValue;
+    const PairArgs a = down_args(rows_cap, offsets, N, d, I, y, status);
     return launch_pair<MODE_DOWN, false>(mr, mw, mt, a, pair_grid(di), st);
+}
+
+cudaError_t launch_grouped_down_e4m3(const void* hq, const float* s_h, int64_t rows_cap,
+                                     const int32_t* offsets, int N, const void* w2q,
+                                     const float* w2_scale, int d, int I, void* y, uint32_t* status,
+                                     cudaStream_t st) {
+    const DevInfo* di = current_device_info();
+    if (!di) return cudaErrorUnknown;
+    CUtensorMap mr, mw, mt;
+    if (!make_tma_map_2d_u8(&mr, hq, static_cast<uint64_t>(rows_cap), I, HALF_M)) return cudaErrorInvalidValue;
+    if (!make_tma_map_2d_u8(&mw, w2q, static_cast<uint64_t>(N) * d, I, HALF_M)) return cudaErrorInvalidValue;
+    if (!make_tma_map_2d_u8(&mt, hq, static_cast<uint64_t>(rows_cap), I, TOK_BOX)) return cudaErrorInvalidValue;
+    PairArgs a = down_args(rows_cap, offsets, N, d, I, y, status);
+    a.row_scale = s_h;
+    a.w_scale = w2_scale;
+    return launch_pair<MODE_DOWN, true>(mr, mw, mt, a, pair_grid(di), st);
 }
 
 }  // namespace lcmoe

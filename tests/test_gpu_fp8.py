@@ -4,9 +4,11 @@ The quantiser is integer-valued work decided in fp32 on both sides (amax, one IE
 the scale, one per element, then round-to-nearest-even to E4M3): codes and scales must match the
 oracle bit for bit. The layer's output is checked with the same rule as the bf16 layer
 (2e-2 x RMS plus half a bf16 step against the oracle's double sums): both sides multiply the
-same E4M3 codes and scales, so they differ only by fp32 accumulation order and the bf16
-roundings of H and Y. The oracle always quantises from the bf16 weights itself; no code or
-scale it uses comes from the GPU.
+same E4M3 codes and scales, so they differ by fp32 accumulation order, the bf16 roundings of H
+and Y, and the E4M3 rounding of an H element that lands next to a rounding boundary. The oracle
+always quantises from the bf16 weights itself; no code or scale it uses comes from the GPU.
+E4M3 K-steps are 128 elements, so the FP8 workloads take I a multiple of 128 (the tiny
+workload's I = 64 is raised to 128).
 """
 import numpy as np
 import pytest
@@ -53,35 +55,39 @@ def test_quantize_ragged_shapes(cuda_device, R, C):
     np.testing.assert_array_equal(q.cpu().numpy(), rq)
 
 
-def oracle_w13(d):
-    """Oracle quantisation of W13 (from the bf16 weights) and its upload for the GPU call."""
+FP8_CHANGES = {"tiny": {"I": 128}, "small": {}}
+
+
+def oracle_weights(d):
+    """Oracle quantisation of W13 and W2 (from the bf16 weights): host arrays and their uploads."""
     w = d["w"]
-    wq, ws = oracle.quantize_rows_e4m3(np_bits(d["w13"]).reshape(w.N * 2 * w.I, w.d))
-    return (wq.reshape(w.N, 2 * w.I, w.d), ws.reshape(w.N, 2 * w.I),
-            torch.from_numpy(wq.reshape(w.N, 2 * w.I, w.d)).cuda(),
-            torch.from_numpy(ws.reshape(w.N, 2 * w.I)).cuda())
+    wq, wsc = oracle.quantize_rows_e4m3(np_bits(d["w13"]).reshape(w.N * 2 * w.I, w.d))
+    w2q, w2s = oracle.quantize_rows_e4m3(np_bits(d["w2"]).reshape(w.N * w.d, w.I))
+    host = (wq.reshape(w.N, 2 * w.I, w.d), wsc.reshape(w.N, 2 * w.I), w2q.reshape(w.N, w.d, w.I),
+            w2s.reshape(w.N, w.d))
+    return host, tuple(torch.from_numpy(a).cuda() for a in host)
 
 
-def forward_fp8(d, w13q, w13s):
+def forward_fp8(d, qw):
     w = d["w"]
     idx = torch.empty(w.T, w.K, dtype=torch.int32, device="cuda")
     gate = torch.empty(w.T, w.K, dtype=torch.float32, device="cuda")
     counts = torch.zeros(w.E, dtype=torch.int32, device="cuda")
     ws = B.new_workspace(B.Shape(w.T, w.d, w.N, w.Z, w.K, w.I), B.OP_FORWARD_FP8)
-    out = B.lc_moe_forward_fp8(d["x"], d["wr"], d["bias"], w13q, w13s, d["w2"], w.K, idx=idx,
-                               gate=gate, counts=counts, ws=ws)
+    out = B.lc_moe_forward_fp8(d["x"], d["wr"], d["bias"], *qw, w.K, idx=idx, gate=gate,
+                               counts=counts, ws=ws)
     assert B.lc_moe_read_status(ws) == 0
     return out, idx, gate, counts
 
 
 @pytest.mark.parametrize("name", ["tiny", "small"])
 def test_forward_fp8_grid_inputs(cuda_device, name):
-    d = make(name, grid=True)
+    d = make(name, grid=True, **FP8_CHANGES[name])
     w = d["w"]
-    wq, wsc, wq_g, wsc_g = oracle_w13(d)
-    out, idx, gate, counts = forward_fp8(d, wq_g, wsc_g)
-    ref = oracle.forward_fp8(np_bits(d["x"]), np_bits(d["wr"]), d["bias"].cpu().numpy(), wq, wsc,
-                             np_bits(d["w2"]), w.N, w.Z, w.K)
+    host, dev = oracle_weights(d)
+    out, idx, gate, counts = forward_fp8(d, dev)
+    ref = oracle.forward_fp8(np_bits(d["x"]), np_bits(d["wr"]), d["bias"].cpu().numpy(), *host,
+                             w.N, w.Z, w.K)
     np.testing.assert_array_equal(idx.cpu().numpy(), ref["idx"])
     np.testing.assert_array_equal(gate.cpu().numpy().view(np.uint32), ref["gate"].view(np.uint32))
     np.testing.assert_array_equal(counts.cpu().numpy(), ref["counts"])
@@ -90,11 +96,11 @@ def test_forward_fp8_grid_inputs(cuda_device, name):
 
 def test_forward_fp8_differs_from_bf16_by_fp8_rounding_only(cuda_device):
     """The FP8 layer and the bf16 layer route identically; their outputs differ by the E4M3
-    rounding of the gate/up operands (a few per cent of the expert terms), not more."""
+    rounding of the expert operands (a few per cent of the expert terms), not more."""
     d = make("small", grid=True)
     w = d["w"]
-    _, _, wq_g, wsc_g = oracle_w13(d)
-    out8, idx8, _, _ = forward_fp8(d, wq_g, wsc_g)
+    _, dev = oracle_weights(d)
+    out8, idx8, _, _ = forward_fp8(d, dev)
     out = B.lc_moe_forward(d["x"], d["wr"], d["bias"], d["w13"], d["w2"], w.K)
     ref_idx = torch.empty_like(idx8)
     B.lc_moe_forward(d["x"], d["wr"], d["bias"], d["w13"], d["w2"], w.K, idx=ref_idx)
@@ -108,7 +114,7 @@ def test_forward_fp8_differs_from_bf16_by_fp8_rounding_only(cuda_device):
 
 def oracle_tokens_fp8(x_bits, tokens, idx, gate, N, w13, w2):
     """Oracle FP8-layer output of the given tokens for the given routing: token rows and the
-    touched experts' W13 quantised by the oracle, one expert at a time."""
+    touched experts' W13 and W2 quantised by the oracle, one expert at a time."""
     K = idx.shape[1]
     d = x_bits.shape[1]
     I = w2.shape[2]
@@ -119,10 +125,11 @@ def oracle_tokens_fp8(x_bits, tokens, idx, gate, N, w13, w2):
     for e in np.unique(experts):
         sel = np.nonzero(experts == e)[0]
         wq, wsc = oracle.quantize_rows_e4m3(np_bits(w13[int(e)]).reshape(2 * I, d))
+        w2q, w2s = oracle.quantize_rows_e4m3(np_bits(w2[int(e)]).reshape(d, I))
         rows = np.array([pairs[i][0] for i in sel])
         _, y = oracle.expert_rows_fp8(np.ascontiguousarray(xq[rows]), np.ascontiguousarray(sx[rows]),
                                       np.zeros(sel.size, np.int32), wq.reshape(1, 2 * I, d),
-                                      wsc.reshape(1, 2 * I), np_bits(w2[int(e)]).reshape(1, d, I),
+                                      wsc.reshape(1, 2 * I), w2q.reshape(1, d, I), w2s.reshape(1, d),
                                       want_h=False)
         Y[sel] = y
     pr = np.full((len(tokens), K), -1, np.int32)
@@ -135,13 +142,14 @@ def oracle_tokens_fp8(x_bits, tokens, idx, gate, N, w13, w2):
 
 @pytest.mark.parametrize("name", ["prefill", "decode"])
 def test_forward_fp8_full_size_sampled(cuda_device, name):
-    """The benchmark's FP8 launch configuration at full size (W13 quantised on the GPU, as the
-    benchmark does), checked on sampled tokens against the oracle's own quantisation."""
+    """The benchmark's FP8 launch configuration at full size (W13 and W2 quantised on the GPU, as
+    the benchmark does), checked on sampled tokens against the oracle's own quantisation."""
     d = make(name)
     w = d["w"]
     w13q, w13s = B.lc_moe_quantize_e4m3(d["w13"])
-    out, idx, gate, _ = forward_fp8(d, w13q, w13s)
-    del w13q, w13s
+    w2q, w2s = B.lc_moe_quantize_e4m3(d["w2"])
+    out, idx, gate, _ = forward_fp8(d, (w13q, w13s, w2q, w2s))
+    del w13q, w13s, w2q, w2s
     rng = np.random.default_rng(17)
     tokens = np.sort(rng.choice(w.T, size=6, replace=False))
     idx_h, gate_h = idx.cpu().numpy(), gate.cpu().numpy()
