@@ -327,7 +327,7 @@ def run_ours(args):
                         "frac": round(ach / peak, 4), "algorithmic_work": work}
     dom = max(STAGES, key=lambda n: stages[n]["ms"])
     ds = stages[dom]
-    trec = None if f8 else traffic_record(dom)
+    trec = traffic_record(dom + ("@fp8" if f8 else ""))
     roofline = {"bound": ds["bound"], "kernel": dom, "achieved": ds["achieved"], "peak": ds["peak"],
                 "unit": ds["unit"], "frac": ds["frac"],
                 "peak_source": (f"{peak_src} ("
