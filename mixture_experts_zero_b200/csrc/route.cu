@@ -70,16 +70,32 @@ __global__ void __launch_bounds__(TOPK_THREADS)
     __syncthreads();
 
     const int warps_total = gridDim.x * (TOPK_THREADS / 32);
-    for (int t = blockIdx.x * (TOPK_THREADS / 32) + warp; t < T; t += warps_total) {
-        const float* zt = logits + static_cast<int64_t>(t) * E;
-        float v[VPL];
-        float m = __int_as_float(0xff800000);  // -inf
+    // up to 32 values per lane (E <= 1024), the next token's logits are loaded while the current
+    // one is processed; above that the registers are needed for the current token
+    constexpr bool PREFETCH = VPL <= 32;
+    float vn[PREFETCH ? VPL : 1];
+    auto load = [&](int tt, float* dst) {
+        const float* zt = logits + static_cast<int64_t>(tt) * E;
 #pragma unroll
         for (int j = 0; j < VPL; ++j) {
             const int i = lane + 32 * j;
-            v[j] = (i < E) ? zt[i] : __int_as_float(0xff800000);
-            m = (v[j] > m) ? v[j] : m;  // a NaN logit is skipped here, and poisons the sum below
+            dst[j] = (tt < T && i < E) ? __ldcs(zt + i) : __int_as_float(0xff800000);
         }
+    };
+    if (PREFETCH) load(blockIdx.x * (TOPK_THREADS / 32) + warp, vn);
+    for (int t = blockIdx.x * (TOPK_THREADS / 32) + warp; t < T; t += warps_total) {
+        float v[VPL];
+        if (PREFETCH) {
+#pragma unroll
+            for (int j = 0; j < VPL; ++j) v[j] = vn[PREFETCH ? j : 0];
+            load(t + warps_total, vn);
+        } else {
+            load(t, v);
+        }
+        float m = __int_as_float(0xff800000);  // -inf
+#pragma unroll
+        for (int j = 0; j < VPL; ++j)
+            m = (v[j] > m) ? v[j] : m;  // a NaN logit is skipped here, and poisons the sum below
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) {
             const float other = __shfl_xor_sync(0xffffffffu, m, o);
