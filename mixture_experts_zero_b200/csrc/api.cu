@@ -154,12 +154,12 @@ int forward_impl(const lc_moe_shape* s, const void* x, const void* wr, const flo
         float* sx = at<float>(ws, L.sx);
         float* s_row = at<float>(ws, L.s_row);
         LC_CUDA(launch_quantize_rows_e4m3(x, s->T, s->d, xq, sx, st));
-        LC_CUDA(launch_gather_e4m3(xq, sx, s->T, s->d, s->K, pair_row, x_perm, s_row, st));
+        LC_CUDA(launch_gather_e4m3(xq, sx, s->T, s->d, s->K, pair_row, x_perm, s_row, status, st));
         LC_TRY(record(events, LC_MOE_STAGE_GEMM1, st));
         LC_CUDA(launch_grouped_swiglu_e4m3(x_perm, s_row, L.rows_cap, offsets, s->N, w13, w13_scale, s->d,
                                            s->I, h, status, st));
     } else {
-        LC_CUDA(launch_gather(x, s->T, s->d, s->K, pair_row, x_perm, st));
+        LC_CUDA(launch_gather(x, s->T, s->d, s->K, pair_row, x_perm, status, st));
         LC_TRY(record(events, LC_MOE_STAGE_GEMM1, st));
         LC_CUDA(launch_grouped_swiglu(x_perm, L.rows_cap, offsets, s->N, w13, s->d, s->I, h, status, st));
     }
@@ -396,7 +396,7 @@ int lc_moe_permute(const lc_moe_shape* s, const int32_t* idx, const void* x, int
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     LC_CUDA(launch_permute(idx, s->T, s->K, s->N, s->N + s->Z, offsets, row_token, pair_row,
                            at<int32_t>(ws, kStatusBytes), at<uint32_t>(ws, 0), st));
-    if (x_perm) LC_CUDA(launch_gather(x, s->T, s->d, s->K, pair_row, x_perm, st));
+    if (x_perm) LC_CUDA(launch_gather(x, s->T, s->d, s->K, pair_row, x_perm, at<uint32_t>(ws, 0), st));
     return LC_MOE_OK;
 }
 
@@ -444,7 +444,7 @@ int lc_moe_permute_noalloc(const lc_moe_shape* s, const int32_t* idx, const void
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     LC_CUDA(launch_permute_noalloc(idx, s->T, s->K, s->N, s->N + s->Z, offsets, row_token, pair_row,
                                    status, st));
-    if (x_perm) LC_CUDA(launch_gather(x, s->T, s->d, s->K, pair_row, x_perm, st));
+    if (x_perm) LC_CUDA(launch_gather(x, s->T, s->d, s->K, pair_row, x_perm, status, st));
     return LC_MOE_OK;
 }
 

@@ -82,6 +82,38 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     }
 }
 
+// ------------------------------------------------------------------------ bulk async copies --
+
+// Contiguous copy global -> shared of `bytes` (multiple of 16, both addresses 16-byte aligned),
+// completion counted on the mbarrier `bar` (no multicast).
+__device__ __forceinline__ void bulk_load_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+// Contiguous copy shared -> global, tracked by this thread's bulk groups.
+__device__ __forceinline__ void bulk_store_s2g(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(dst), "r"(smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+// Order this thread's view of shared memory (including copies it waited for) before later
+// async-proxy accesses (bulk copies, TMA, tensor-core operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's bulk groups are still reading their shared memory source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until at most N of this thread's bulk groups are still in flight.
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ------------------------------------------------------------------------------------- TMA --
 
 // 2-D tiled bulk-tensor load global -> shared, completion counted on `bar` (no multicast).
@@ -340,11 +372,12 @@ cudaError_t launch_permute(const int32_t* idx, int T, int K, int N, int E, int32
                            int32_t* row_token, int32_t* pair_row, int32_t* scratch,
                            uint32_t* status, cudaStream_t st);
 cudaError_t launch_gather(const void* x, int T, int d, int K, const int32_t* pair_row,
-                          void* x_perm, cudaStream_t st);
+                          void* x_perm, uint32_t* status, cudaStream_t st);
 // Row gather of E4M3 token rows (d bytes each) with their scales: x_perm[pair_row[t,k]] = xq[t],
 // s_row[pair_row[t,k]] = sx[t].
 cudaError_t launch_gather_e4m3(const void* xq, const float* sx, int T, int d, int K,
-                               const int32_t* pair_row, void* x_perm, float* s_row, cudaStream_t st);
+                               const int32_t* pair_row, void* x_perm, float* s_row, uint32_t* status,
+                               cudaStream_t st);
 
 // Row-wise E4M3 quantisation of a bf16 matrix [R, C] (C % 8 == 0): scale[r] = amax / 448
 // (1 for an all-zero row), dst[r, c] = E4M3(src[r, c] / scale[r]) (round to nearest even,

@@ -188,6 +188,126 @@ __global__ void __launch_bounds__(GATHER_THREADS)
     }
 }
 
+// Row gather with bulk async copies: warp w of a block owns two shared-memory row slots. Its
+// first lane loads token t's row with one cp.async.bulk (completion on the slot's mbarrier), and
+// once it has landed writes it to each of the token's FFN rows with one bulk store per row; the
+// next token's row is loaded into the other slot meanwhile, after the stores that last read
+// that slot are done reading it. The copies never pass through registers. Every wait is bounded
+// (LC_MOE_DEV_WAIT_TIMEOUT).
+constexpr int GB_WARPS = 4;
+constexpr uint32_t GB_MAX_ROW_BYTES = 25600;  // 2 slots x 4 warps within 200 KB of shared memory
+
+__global__ void __launch_bounds__(GB_WARPS * 32)
+    gather_bulk_kernel(const uint8_t* __restrict__ x, int T, uint32_t row_bytes, int K,
+                       const int32_t* __restrict__ pair_row, uint8_t* __restrict__ x_perm,
+                       const float* __restrict__ sx, float* __restrict__ s_row, uint32_t* status,
+                       uint64_t wait_ns) {
+    extern __shared__ __align__(128) uint8_t gsm[];
+    __shared__ uint64_t bars[GB_WARPS][2];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t* slot0 = gsm + static_cast<size_t>(2 * warp) * row_bytes;
+    uint8_t* slot1 = slot0 + row_bytes;
+    if (lane == 0) {
+        mbar_init(&bars[warp][0], 1);
+        mbar_init(&bars[warp][1], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    const int stride = gridDim.x * GB_WARPS;
+    int t = blockIdx.x * GB_WARPS + warp;
+    uint32_t ph0 = 0, ph1 = 0;
+    int b = 0;
+    if (lane == 0 && t < T) {
+        mbar_arrive_expect_tx(&bars[warp][0], row_bytes);
+        bulk_load_g2s(slot0, x + static_cast<int64_t>(t) * row_bytes, row_bytes, &bars[warp][0]);
+    }
+    for (; t < T; t += stride) {
+        const int tn = t + stride;
+        const int my_row = (lane < K) ? pair_row[static_cast<int64_t>(t) * K + lane] : -1;
+        if (s_row && my_row >= 0) s_row[my_row] = sx[t];  // row scale of E4M3 rows
+        const uint32_t dests = __ballot_sync(0xffffffffu, my_row >= 0);
+        uint8_t* cur = b ? slot1 : slot0;
+        uint8_t* nxt = b ? slot0 : slot1;
+        int got = 1;
+        if (lane == 0) {
+            const bool nxt_issued = tn < T;
+            if (nxt_issued) {
+                // the stores issued from the other slot (previous token) must be done reading it
+                bulk_wait_read<0>();
+                mbar_arrive_expect_tx(&bars[warp][b ^ 1], row_bytes);
+                bulk_load_g2s(nxt, x + static_cast<int64_t>(tn) * row_bytes, row_bytes, &bars[warp][b ^ 1]);
+            }
+            const uint32_t ph = b ? ph1 : ph0;
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&bars[warp][b], ph)) {
+                if (globaltimer_ns() - t0 > wait_ns) {
+                    set_status(status, LC_MOE_DEV_WAIT_TIMEOUT);
+                    got = 0;
+                    break;
+                }
+            }
+            if (got) {
+                fence_proxy_async_smem();
+            } else if (nxt_issued) {
+                // do not leave while the other slot's load may still be writing it
+                const uint32_t phn = b ? ph0 : ph1;
+                const uint64_t t1 = globaltimer_ns();
+                while (!mbar_try_wait(&bars[warp][b ^ 1], phn) && globaltimer_ns() - t1 < wait_ns) {
+                }
+            }
+        }
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) break;
+        if (b) ph1 ^= 1u;
+        else ph0 ^= 1u;
+        uint32_t m = dests;
+        while (m) {
+            const int r = __ffs(m) - 1;
+            m &= m - 1;
+            const int row = __shfl_sync(0xffffffffu, my_row, r);
+            if (lane == 0) bulk_store_s2g(x_perm + static_cast<int64_t>(row) * row_bytes, cur, row_bytes);
+        }
+        if (lane == 0) bulk_commit();
+        b ^= 1;
+    }
+    if (lane == 0) bulk_wait<0>();  // the last stores have left shared memory and landed
+}
+
+cudaError_t launch_gather_rows(const void* x, int T, uint32_t row_bytes, int K, const int32_t* pair_row,
+                               void* x_perm, const float* sx, float* s_row, uint32_t* status,
+                               cudaStream_t st) {
+    const DevInfo* di = current_device_info();
+    if (!di) return cudaErrorUnknown;
+    if (T == 0) return cudaSuccess;
+    if (row_bytes <= GB_MAX_ROW_BYTES) {
+        const size_t smem = static_cast<size_t>(2 * GB_WARPS) * row_bytes;
+        static int configured[64] = {0};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 64 && !configured[dev]) {
+            e = cudaFuncSetAttribute(gather_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(2 * GB_WARPS * GB_MAX_ROW_BYTES));
+            if (e != cudaSuccess) return e;
+            configured[dev] = 1;
+        }
+        int blocks = (T + GB_WARPS - 1) / GB_WARPS;
+        const int per_sm = smem ? static_cast<int>((200u * 1024u) / smem) : 8;
+        const int cap = di->sm_count * (per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm));
+        if (blocks > cap) blocks = cap;
+        gather_bulk_kernel<<<blocks, GB_WARPS * 32, smem, st>>>(static_cast<const uint8_t*>(x), T, row_bytes, K,
+                                                                 pair_row, static_cast<uint8_t*>(x_perm), sx,
+                                                                 s_row, status, wait_limit_ns());
+        return cudaGetLastError();
+    }
+    const int warps = GATHER_THREADS / 32;
+    int blocks = (T + warps - 1) / warps;
+    if (blocks > di->sm_count * 8) blocks = di->sm_count * 8;
+    gather_kernel<<<blocks, GATHER_THREADS, 0, st>>>(static_cast<const uint4*>(x), T, static_cast<int>(row_bytes / 16),
+                                                      K, pair_row, static_cast<uint4*>(x_perm), sx, s_row);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t permute_scratch_bytes(int T, int N) {
@@ -228,29 +348,15 @@ cudaError_t launch_permute(const int32_t* idx, int T, int K, int N, int E, int32
 }
 
 cudaError_t launch_gather(const void* x, int T, int d, int K, const int32_t* pair_row, void* x_perm,
-                          cudaStream_t st) {
-    const DevInfo* di = current_device_info();
-    if (!di) return cudaErrorUnknown;
-    if (T == 0) return cudaSuccess;
-    const int warps = GATHER_THREADS / 32;
-    int blocks = (T + warps - 1) / warps;
-    if (blocks > di->sm_count * 8) blocks = di->sm_count * 8;
-    gather_kernel<<<blocks, GATHER_THREADS, 0, st>>>(static_cast<const uint4*>(x), T, d / 8, K, pair_row,
-                                                      static_cast<uint4*>(x_perm), nullptr, nullptr);
-    return cudaGetLastError();
+                          uint32_t* status, cudaStream_t st) {
+    return launch_gather_rows(x, T, static_cast<uint32_t>(d) * 2, K, pair_row, x_perm, nullptr, nullptr,
+                              status, st);
 }
 
 cudaError_t launch_gather_e4m3(const void* xq, const float* sx, int T, int d, int K,
-                               const int32_t* pair_row, void* x_perm, float* s_row, cudaStream_t st) {
-    const DevInfo* di = current_device_info();
-    if (!di) return cudaErrorUnknown;
-    if (T == 0) return cudaSuccess;
-    const int warps = GATHER_THREADS / 32;
-    int blocks = (T + warps - 1) / warps;
-    if (blocks > di->sm_count * 8) blocks = di->sm_count * 8;
-    gather_kernel<<<blocks, GATHER_THREADS, 0, st>>>(static_cast<const uint4*>(xq), T, d / 16, K, pair_row,
-                                                      static_cast<uint4*>(x_perm), sx, s_row);
-    return cudaGetLastError();
+                               const int32_t* pair_row, void* x_perm, float* s_row, uint32_t* status,
+                               cudaStream_t st) {
+    return launch_gather_rows(xq, T, static_cast<uint32_t>(d), K, pair_row, x_perm, sx, s_row, status, st);
 }
 
 // ---------------------------------------------------------------------------------------------
