@@ -119,13 +119,13 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------- our arm ----
 
-def traffic_record(peaks_kernel: str):
+def traffic_record(key: str):
     """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if it was taken
     on the current kernel source."""
     p = ROOT / "profiles" / "traffic.json"
     if not p.exists():
         return None
-    rec = json.loads(p.read_text()).get(peaks_kernel)
+    rec = json.loads(p.read_text()).get(key)
     if not rec:
         return None
     src = ROOT / "mixture_experts_zero_b200" / "csrc" / rec["source"]
@@ -327,7 +327,7 @@ def run_ours(args):
                         "frac": round(ach / peak, 4), "algorithmic_work": work}
     dom = max(STAGES, key=lambda n: stages[n]["ms"])
     ds = stages[dom]
-    trec = traffic_record(dom + ("@fp8" if f8 else ""))
+    trec = traffic_record(f"{w.name}/{dom}" + ("@fp8" if f8 else ""))
     roofline = {"bound": ds["bound"], "kernel": dom, "achieved": ds["achieved"], "peak": ds["peak"],
                 "unit": ds["unit"], "frac": ds["frac"],
                 "peak_source": (f"{peak_src} ("
