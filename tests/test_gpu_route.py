@@ -124,3 +124,52 @@ def test_nan_logits_set_the_device_status(cuda_device):
     assert status & B.DEV_NAN_KEY
     assert idx[2].cpu().tolist() == [0, 1, 2] and torch.isnan(gate[2]).all()
     assert B.lc_moe_read_status(ws) == 0  # cleared
+
+
+# (T, d, E, K): expert counts below, at and between multiples of the router GEMM's 256-wide N
+# tile and of 32 (the top-K kernel's lane stride), ragged token counts past a 128-row M tile,
+# K = 1 and K = 16, with frequent exact ties (small d, integer-grid inputs)
+ROUTE_SHAPES = [(64, 128, 12, 3), (257, 64, 96, 6), (1, 64, 300, 12), (300, 128, 512, 16),
+                (513, 64, 700, 12), (1000, 256, 768, 12), (129, 64, 768, 1), (70, 64, 33, 16)]
+
+
+@pytest.mark.parametrize("shape", ROUTE_SHAPES, ids=[str(s) for s in ROUTE_SHAPES])
+def test_route_without_logits_buffer_bit_exact_on_grid_inputs(cuda_device, shape):
+    """lc_moe_route with the logits kept in its workspace: on grid inputs its picks, gates and
+    counts equal the oracle's routing of the exact logits."""
+    T, d, E, K = shape
+    g = torch.Generator(device="cuda").manual_seed(T * 7 + E)
+    x = inputs.to_grid(torch.randn(T, d, generator=g, device="cuda") * 2)
+    wr = (torch.randint(-4, 5, (E, d), generator=g, device="cuda").float() * 2.0 ** -6).to(torch.bfloat16)
+    bias = (torch.randint(-2, 3, (E,), generator=g, device="cuda").float() * 2.0 ** -9)
+    N = max(1, (2 * E) // 3)
+    counts = torch.zeros(E, dtype=torch.int32, device="cuda")
+    ws = B.new_workspace(B.Shape(T, d, N, E - N, K, 64), B.OP_ROUTE)
+    idx, gate = B.lc_moe_route(x, wr, bias, K, N, counts=counts, ws=ws)
+    assert B.lc_moe_read_status(ws) == 0
+    z = oracle.router_logits(np_bits(x), np_bits(wr))
+    np.testing.assert_array_equal(z, exact_grid_logits(x, wr))
+    r_idx, r_gate, r_counts, bad = oracle.route(z, bias.cpu().numpy(), K)
+    assert bad == 0
+    np.testing.assert_array_equal(idx.cpu().numpy(), r_idx)
+    np.testing.assert_array_equal(gate.cpu().numpy().view(np.uint32), r_gate.view(np.uint32))
+    np.testing.assert_array_equal(counts.cpu().numpy(), r_counts)
+
+
+@pytest.mark.parametrize("name", ["decode", "prefill"])
+def test_route_full_shape_grid_inputs(cuda_device, name):
+    """LongCat-Flash shape on grid activations: the router logits are exact in any summation order
+    (checked against an int64 product on sampled rows), so lc_moe_route's routing of every token
+    must equal the oracle's routing of those exact logits, bit for bit."""
+    d = make(name, grid=True, experts=False)
+    w = d["w"]
+    counts = torch.zeros(w.E, dtype=torch.int32, device="cuda")
+    idx, gate = B.lc_moe_route(d["x"], d["wr"], d["bias"], w.K, w.N, counts=counts)
+    z = B.lc_moe_router_logits(d["x"], d["wr"])
+    rows = np.arange(0, w.T, max(1, w.T // 16))
+    np.testing.assert_array_equal(z.cpu().numpy()[rows], exact_grid_logits(d["x"][rows], d["wr"]))
+    r_idx, r_gate, r_counts, bad = oracle.route(z.cpu().numpy(), d["bias"].cpu().numpy(), w.K)
+    assert bad == 0
+    np.testing.assert_array_equal(idx.cpu().numpy(), r_idx)
+    np.testing.assert_array_equal(gate.cpu().numpy().view(np.uint32), r_gate.view(np.uint32))
+    np.testing.assert_array_equal(counts.cpu().numpy(), r_counts)
