@@ -40,6 +40,16 @@ KERNELS_PER_STAGE = (1, 1, 3, 1, 1, 1, 1)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def load_peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -438,6 +448,7 @@ def cpu_baseline(w, data, budget_s: float = 20.0):
         if spent < budget_s / 4:
             n = min(n * 2, 64)
     return {"value": round(tok / spent, 3), "unit": UNIT, "cores": oracle.num_threads(),
+            "cpu": cpu_model(), "host_cpus": os.cpu_count(),
             "kind": "oracle",
             "sample": f"{int(tok)} random tokens of the {w.name} batch (router logits, routing, "
                       f"SwiGLU experts of their FFN picks, combine), {spent:.1f} s of oracle time; "
@@ -491,6 +502,7 @@ def run_reference(args):
                    "d": w.d, "N": w.N, "Z": w.Z, "K": w.K, "K_e": w.K_e, "I": w.I,
                    "router": w.router, "parallelism": "none (host cores)"},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.num_threads(),
+                         "cpu": cpu_model(), "host_cpus": os.cpu_count(),
                          "kind": "oracle",
                          "sample": f"{per_step_tokens} fresh tokens per step of the {w.name} workload"},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
