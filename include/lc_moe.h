@@ -33,6 +33,9 @@
  *     lc_moe_read_status clears it. Calls that share a workspace must be ordered on one stream.
  *   - Host-side checks run before any launch; a failing check returns a status code and
  *     enqueues nothing. Functions never abort, throw or print.
+ *   - Every entry point except lc_moe_read_status can be captured in a CUDA graph once it has
+ *     been called on the device outside a capture (the first call sets kernel attributes and
+ *     looks up the driver's tensor-map encoder).
  *   - Shape limits (else LC_MOE_ERR_UNSUPPORTED_SHAPE): d and I multiples of 64 and >= 64;
  *     1 <= K <= 32; K <= N+Z <= 2048; N >= 1; Z >= 0; T >= 0; T*K < 2^31. T = 0 is a no-op.
  */
