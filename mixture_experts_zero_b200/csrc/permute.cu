@@ -13,8 +13,10 @@
 //   scatter : the row of pick (t, r) of expert e is
 //             offsets[e] + base[b][e] + popc(mask of e restricted to tokens before t in block b),
 //             so rows of an expert are in ascending token order. Writes pair_row and row_token.
-//   gather  : one warp per token copies x_t (16-byte vectors) to each of its FFN rows; x_t is
-//             read once however many FFN experts the token picked.
+//   gather  : per token, x_t is read once into shared memory with one bulk async copy and
+//             written to each of its FFN rows with one bulk store per row (rows above 25 KB:
+//             one warp per token copies 16-byte vectors through registers); x_t is read once
+//             however many FFN experts the token picked.
 #include <mutex>
 
 #include "common.cuh"

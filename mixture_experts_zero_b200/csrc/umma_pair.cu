@@ -25,16 +25,16 @@
 //   row tiles: 256 rows of one expert. GEMM 1: the leader loads 128 gate rows and its peer the
 //     matching 128 up rows of B, so accumulator columns [0, 128) hold gate and [128, 256) hold up
 //     values for every row. GEMM 2: 256 output features, 128 per CTA.
-//   weight tiles ("swap"): 256 weight rows (128 per CTA) on the M side and up to 256 rows of one
-//     expert, rounded up to 64 and split between the CTAs, on the N side. GEMM 1 issues a gate MMA
-//     into columns [0, N) and an up MMA into [128, 128 + N) (N <= 128).
+//   weight tiles ("swap"): 256 weight rows (128 per CTA) on the M side and the rows of one expert,
+//     rounded up to 64 and split between the CTAs, on the N side (N <= 128 for GEMM 1, <= 256 for
+//     GEMM 2). GEMM 1 issues a gate MMA into columns [0, N) and an up MMA into [128, 128 + N).
 // Per expert with c_e rows: below cold_rows it is "cold" and runs as weight tiles only; otherwise
 // it runs floor(c_e / 256) row tiles, and its leftover rows run as one more row tile if there are
-// at least rem_rows of them, else as weight tiles (N rounded up to 64): an expert's padding rows
-// stay below 128 for GEMM 1 (rem_rows = 128) and below 64 for GEMM 2 (rem_rows = 256). The tile list (built on the device from offsets, identically
-// by every CTA) is: for each hot expert in order, its row tiles then its leftover weight tiles
-// (whose weights were just read by its row tiles and are still in L2); then the weight tiles of
-// every cold expert. Tile t goes to cluster t mod (gridDim / 2).
+// at least rem_rows of them, else as weight tiles (N rounded up to 64). GEMM 1: cold_rows =
+// rem_rows = 128; GEMM 2: cold_rows = rem_rows = 256. The tile list (built on the device from
+// offsets, identically by every CTA) is: for each hot expert in order, its row tiles then its
+// leftover weight tiles; then the weight tiles of every cold expert. Tile t goes to cluster
+// t mod (gridDim / 2).
 // Every wait is bounded (lc_moe_set_wait_limit_ns); a wait that runs out raises a CTA-wide abort,
 // records LC_MOE_DEV_WAIT_TIMEOUT, drains in-flight copies and MMAs, and frees TMEM.
 #include <cudaTypedefs.h>
