@@ -31,13 +31,19 @@ __device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
 }
 
+// Work item = (token, column block): a warp handles `span` 16-byte chunks of one token's row
+// (all of it for large T; several warps share a row when T is too small to fill the GPU).
 __global__ void __launch_bounds__(COMBINE_THREADS)
     combine_kernel(const uint4* __restrict__ x, const uint4* __restrict__ y,
                    const float* __restrict__ gate, const int32_t* __restrict__ pair_row, int T,
-                   int d8, int K, uint4* __restrict__ out) {
+                   int d8, int K, int cb, int span, uint4* __restrict__ out) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (COMBINE_THREADS / 32);
-    for (int t = blockIdx.x * (COMBINE_THREADS / 32) + warp; t < T; t += warps_total) {
+    const int items = T * cb;  // cb > 1 only while T * cb stays near the warp count of one wave
+    for (int it = blockIdx.x * (COMBINE_THREADS / 32) + warp; it < items; it += warps_total) {
+        const int t = cb == 1 ? it : it / cb;
+        const int c_begin = (it - t * cb) * span;
+        const int c_end = min(d8, c_begin + span);
         float my_g = 0.0f;
         int my_row = -1;
         if (lane < K) {
@@ -46,13 +52,13 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
         }
         const bool any_zero = __any_sync(0xffffffffu, lane < K && my_row < 0);
         const uint4* xt = x + static_cast<int64_t>(t) * d8;
-        for (int c0 = 0; c0 < d8; c0 += 64) {  // warp-uniform trip count
-            const int ca = c0 + lane, cb = c0 + 32 + lane;
-            const bool ina = ca < d8, inb = cb < d8;
+        for (int c0 = c_begin; c0 < c_end; c0 += 64) {  // warp-uniform trip count
+            const int ca = c0 + lane, cb2 = c0 + 32 + lane;
+            const bool ina = ca < c_end, inb = cb2 < c_end;
             uint4 xa = make_uint4(0, 0, 0, 0), xb = xa;
             if (any_zero) {
                 if (ina) xa = __ldg(xt + ca);
-                if (inb) xb = __ldg(xt + cb);
+                if (inb) xb = __ldg(xt + cb2);
             }
             float acc_a[8], acc_b[8];
 #pragma unroll
@@ -71,7 +77,7 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
                     const bool pick = r0 + u < K;
                     const uint4* yr = y + static_cast<int64_t>(row[u] < 0 ? 0 : row[u]) * d8;
                     va[u] = (pick && row[u] >= 0 && ina) ? __ldg(yr + ca) : xa;
-                    vb[u] = (pick && row[u] >= 0 && inb) ? __ldg(yr + cb) : xb;
+                    vb[u] = (pick && row[u] >= 0 && inb) ? __ldg(yr + cb2) : xb;
                 }
                 // rank order: pick r0, r0 + 1, ... each one fused multiply-add per element
 #pragma unroll
@@ -83,7 +89,7 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
                 }
             }
             if (ina) out[static_cast<int64_t>(t) * d8 + ca] = pack8(acc_a);
-            if (inb) out[static_cast<int64_t>(t) * d8 + cb] = pack8(acc_b);
+            if (inb) out[static_cast<int64_t>(t) * d8 + cb2] = pack8(acc_b);
         }
     }
 }
@@ -97,11 +103,20 @@ cudaError_t launch_combine(const void* x, const void* y, const float* gate,
     if (!di) return cudaErrorUnknown;
     if (T == 0) return cudaSuccess;
     const int warps = COMBINE_THREADS / 32;
-    int blocks = (T + warps - 1) / warps;
+    const int d8 = d / 8;
+    // column blocks per token: enough (token, block) items for 8 blocks of 8 warps per SM
+    const int max_cb = (d8 + 63) / 64;
+    int cb = (di->sm_count * 8 * warps + T - 1) / T;
+    if (cb > max_cb) cb = max_cb;
+    if (cb < 1) cb = 1;
+    const int span = ((d8 + cb - 1) / cb + 63) / 64 * 64;
+    cb = (d8 + span - 1) / span;
+    const int64_t items = static_cast<int64_t>(T) * cb;
+    int64_t blocks = (items + warps - 1) / warps;
     if (blocks > di->sm_count * 8) blocks = di->sm_count * 8;
-    combine_kernel<<<blocks, COMBINE_THREADS, 0, st>>>(static_cast<const uint4*>(x),
-                                                        static_cast<const uint4*>(y), gate, pair_row,
-                                                        T, d / 8, K, static_cast<uint4*>(out));
+    combine_kernel<<<static_cast<int>(blocks), COMBINE_THREADS, 0, st>>>(
+        static_cast<const uint4*>(x), static_cast<const uint4*>(y), gate, pair_row, T, d8, K, cb, span,
+        static_cast<uint4*>(out));
     return cudaGetLastError();
 }
 

@@ -285,6 +285,10 @@ cudaError_t launch_router_gemm(const void* x, const void* wr, float* logits, int
     if (!di) return cudaErrorUnknown;
     int bn = ((E + 31) / 32) * 32;
     if (bn > 256) bn = 256;
+    // few token tiles (decode-sized T): narrower expert tiles, down to 32, so that more SMs
+    // stream the router weight
+    const int m_tiles = (T + BM - 1) / BM;
+    while (bn > 32 && m_tiles * ((E + bn - 1) / bn) < di->sm_count) bn = ((bn / 2 + 31) / 32) * 32;
     CUtensorMap ma, mb;
     if (!make_tma_map_2d(&ma, x, static_cast<uint64_t>(T), d, BM)) return cudaErrorInvalidValue;
     if (!make_tma_map_2d(&mb, wr, static_cast<uint64_t>(E), d, bn)) return cudaErrorInvalidValue;
