@@ -31,19 +31,20 @@ __device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
 }
 
-// Work item = (token, column block): a warp handles `span` 16-byte chunks of one token's row
-// (all of it for large T; several warps share a row when T is too small to fill the GPU).
+// Work item: one token's row (SPLIT = false), or a (token, column block) of `span` 16-byte chunks
+// (SPLIT = true, when T is too small for one warp per token to fill the GPU).
+template <bool SPLIT>
 __global__ void __launch_bounds__(COMBINE_THREADS)
     combine_kernel(const uint4* __restrict__ x, const uint4* __restrict__ y,
                    const float* __restrict__ gate, const int32_t* __restrict__ pair_row, int T,
                    int d8, int K, int cb, int span, uint4* __restrict__ out) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int warps_total = gridDim.x * (COMBINE_THREADS / 32);
-    const int items = T * cb;  // cb > 1 only while T * cb stays near the warp count of one wave
+    const int items = SPLIT ? T * cb : T;  // T * cb stays near the warp count of one wave
     for (int it = blockIdx.x * (COMBINE_THREADS / 32) + warp; it < items; it += warps_total) {
-        const int t = cb == 1 ? it : it / cb;
-        const int c_begin = (it - t * cb) * span;
-        const int c_end = min(d8, c_begin + span);
+        const int t = SPLIT ? it / cb : it;
+        const int c_begin = SPLIT ? (it - t * cb) * span : 0;
+        const int c_end = SPLIT ? min(d8, c_begin + span) : d8;
         float my_g = 0.0f;
         int my_row = -1;
         if (lane < K) {
@@ -114,9 +115,14 @@ cudaError_t launch_combine(const void* x, const void* y, const float* gate,
     const int64_t items = static_cast<int64_t>(T) * cb;
     int64_t blocks = (items + warps - 1) / warps;
     if (blocks > di->sm_count * 8) blocks = di->sm_count * 8;
-    combine_kernel<<<static_cast<int>(blocks), COMBINE_THREADS, 0, st>>>(
-        static_cast<const uint4*>(x), static_cast<const uint4*>(y), gate, pair_row, T, d8, K, cb, span,
-        static_cast<uint4*>(out));
+    if (cb > 1)
+        combine_kernel<true><<<static_cast<int>(blocks), COMBINE_THREADS, 0, st>>>(
+            static_cast<const uint4*>(x), static_cast<const uint4*>(y), gate, pair_row, T, d8, K, cb, span,
+            static_cast<uint4*>(out));
+    else
+        combine_kernel<false><<<static_cast<int>(blocks), COMBINE_THREADS, 0, st>>>(
+            static_cast<const uint4*>(x), static_cast<const uint4*>(y), gate, pair_row, T, d8, K, 1, d8,
+            static_cast<uint4*>(out));
     return cudaGetLastError();
 }
 
