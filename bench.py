@@ -50,6 +50,19 @@ def cpu_model() -> str:
     return "unknown"
 
 
+def workload_config(w, world: int, f8: bool) -> dict:
+    """The `config` of both arms' JSON line for workload w on `world` ranks."""
+    return {"workload": f"{w.name}: MoE layer with zero-computation experts, T={w.T} tokens per GPU",
+            "T": w.T, "d": w.d, "N": w.N, "Z": w.Z, "K": w.K, "K_e": w.K_e, "I": w.I,
+            "router": w.router, "mu": w.mu, "parallelism": f"dp{world}",
+            "step": "forward + counts all-reduce (N>1) + expert-bias update",
+            "experts": ("all expert projections on E4M3 codes with one fp32 scale per weight "
+                        "row and per activation row (weights quantised once before timing)")
+                       if f8 else "bf16",
+            "l2": f"inputs larger than L2 ({w.weight_bytes() / 1e9:.1f} GB expert weights, "
+                  f"{w.T * w.d * 2 / 1e6:.0f} MB x per step)"}
+
+
 def load_peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -358,15 +371,7 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3 experts + bf16 router/combine" if f8 else "bf16",
         "data": "synthetic (seeded; random-init weights of the LongCat-Flash MoE-layer shape)",
-        "config": {"workload": f"{w.name}: MoE layer with zero-computation experts, T={T} tokens per GPU",
-                   "T": T, "d": d_, "N": w.N, "Z": w.Z, "K": K, "K_e": w.K_e, "I": I_,
-                   "router": w.router, "mu": w.mu, "parallelism": f"dp{world}",
-                   "step": "forward + counts all-reduce (N>1) + expert-bias update",
-                   "experts": ("all expert projections on E4M3 codes with one fp32 scale per weight "
-                               "row and per activation row (weights quantised once before timing)")
-                              if f8 else "bf16",
-                   "l2": f"inputs larger than L2 ({w.weight_bytes() / 1e9:.1f} GB expert weights, "
-                         f"{T * d_ * 2 / 1e6:.0f} MB x per step)"},
+        "config": workload_config(w, world, f8),
         "roofline": roofline,
         "layer_roofline": {"t_roof_ms": round(t_roof * 1e3, 4), "frac": round(t_roof * 1e3 / ms_per_step, 4),
                            "alg_flop": flops, "alg_bytes": bytes_, "ffn_rows_M": M,
@@ -498,9 +503,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_s / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name}: LongCat-Flash-shape MoE layer, prefill batch", "T": w.T,
-                   "d": w.d, "N": w.N, "Z": w.Z, "K": w.K, "K_e": w.K_e, "I": w.I,
-                   "router": w.router, "parallelism": "none (host cores)"},
+        "config": workload_config(w, int(os.environ.get("WORLD_SIZE", "1")), False),
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.num_threads(),
                          "cpu": cpu_model(), "host_cpus": os.cpu_count(),
                          "kind": "oracle",
