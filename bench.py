@@ -526,9 +526,14 @@ def run_sweep(args):
     ffn_rows: the two grouped expert GEMMs (lc_moe_expert_ffn) at the prefill shape (d=6144,
         I=2048) with c rows for each of n experts, against max(6*M*d*I FLOP / sustained TC peak,
         (3*n*d*I + 2*M*(2d+I)) * 2 bytes / HBM).
-    hist: the expert-count histogram over idx[2^24, 12] (805 MB of int32), against HBM."""
+    hist: the expert-count histogram over idx[2^24, 12] (805 MB of int32), against HBM.
+    control: the bias-control loop at LongCat-Flash shape (run_control)."""
     import torch
     from mixture_experts_zero_b200 import binding as B
+
+    if args.sweep == "control":
+        run_control(args)
+        return
 
     peaks, peak_src = load_peaks()
     dev = torch.device("cuda", 0)
@@ -587,6 +592,70 @@ def run_sweep(args):
         del x, h, y
 
 
+def run_control(args):
+    """The bias-control loop at LongCat-Flash shape (T = 8192 fresh N(0,1) tokens per step,
+    d = 6144, 512 FFN + 256 zero experts, K = 12, K_e = 8, 200 steps): each step routes on the
+    device (lc_moe_route: router GEMM, softmax + biased top-K, expert counts) and applies
+    b_i += mu (K_e/(K N) - T_i/(K T_all)) (lc_moe_bias_update). One JSON line per (start, mu):
+    the mean number of FFN experts per token every 10 steps, the expert-load spread
+    max_i T_i / mean_i T_i at the first and last step, and the device time of one control step
+    (route + update, CUDA events; drawing the tokens is outside it). Starts: b = 0, and b = +2/E
+    on the zero experts (routing pushed toward the zero experts, below K_e FFN experts per token).
+    mu = 1e-3 is the workload's; the larger mu show the direction and speed of the control within
+    200 steps, since at 1e-3 the pages' convergence needs orders of magnitude more tokens."""
+    import torch
+    from mixture_experts_zero_b200 import binding as B
+    from mixture_experts_zero_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = inputs.WORKLOADS["bias_loop"]
+    s = B.Shape(w.T, w.d, w.N, w.Z, w.K, w.I)
+    ws = B.new_workspace(s, B.OP_ROUTE, dev)
+    idx = torch.empty(w.T, w.K, dtype=torch.int32, device=dev)
+    gate = torch.empty(w.T, w.K, dtype=torch.float32, device=dev)
+    counts = torch.zeros(w.E, dtype=torch.int32, device=dev)
+    for start in ("zero", "zero_experts_favoured"):
+        for mu in (1e-3, 1e-2, 1e-1):
+            g = inputs.generator(w.seed, dev)
+            wr = inputs.draw_router(w, g, dev)
+            bias = torch.zeros(w.E, dtype=torch.float32, device=dev)
+            if start != "zero":
+                bias[w.N:] = 2.0 / w.E
+            ffn = torch.zeros(w.steps, dtype=torch.int64, device=dev)
+            spread = torch.zeros(w.steps, dtype=torch.float64, device=dev)
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                   torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(w.steps)]
+            counts.zero_()
+            for step in range(w.steps):
+                x = inputs.draw_x(w, g, dev)
+                e0, e1, e2, e3 = ev[step]
+                e0.record()
+                B.lc_moe_route(x, wr, bias, w.K, w.N, idx=idx, gate=gate, counts=counts, ws=ws)
+                e1.record()
+                ffn[step] = counts[: w.N].sum()
+                spread[step] = counts.max().double() / (w.T * w.K / w.E)
+                e2.record()
+                B.lc_moe_bias_update(bias, counts, w.T, w.N, w.Z, w.K, w.K_e, mu, reset_counts=True)
+                e3.record()
+            torch.cuda.synchronize()
+            B.lc_moe_read_status(ws)
+            ms = sorted(a.elapsed_time(b) + c.elapsed_time(d) for a, b, c, d in ev)
+            mean_ffn = (ffn.double() / w.T).cpu().tolist()
+            sp = spread.cpu().tolist()
+            zero_bias = bias[w.N:].mean().item() - bias[: w.N].mean().item()
+            print(json.dumps({
+                "sweep": "control", "workload": f"bias_loop: T={w.T} fresh tokens per step, "
+                f"d={w.d}, N={w.N}, Z={w.Z}, K={w.K}, K_e={w.K_e}", "steps": w.steps, "mu": mu,
+                "start": start, "mean_ffn_per_token_every_10": [round(v, 4) for v in mean_ffn[::10]],
+                "mean_ffn_per_token_last": round(mean_ffn[-1], 4),
+                "mean_ffn_per_token_last10": round(sum(mean_ffn[-10:]) / 10, 4),
+                "load_max_over_mean_first_last": [round(sp[0], 3), round(sp[-1], 3)],
+                "zero_minus_ffn_mean_bias": zero_bias,
+                "control_step_ms_median": round(ms[len(ms) // 2], 4)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -600,7 +669,7 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=4, help="tokens per reference-arm step")
     ap.add_argument("--experts", choices=["bf16", "fp8"], default="bf16",
                     help="fp8: E4M3 expert projections (lc_moe_forward_fp8)")
-    ap.add_argument("--sweep", choices=["ffn_rows", "hist"], default=None,
+    ap.add_argument("--sweep", choices=["ffn_rows", "hist", "control"], default=None,
                     help="run a kernel sweep instead of the step (one GPU)")
     args = ap.parse_args()
     if args.sweep:
