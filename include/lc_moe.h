@@ -111,6 +111,15 @@ size_t lc_moe_workspace_bytes(const lc_moe_shape* s, int op);
  * returns early with partial results. Values below 1e6 are raised to 1e6. */
 void lc_moe_set_wait_limit_ns(uint64_t limit_ns);
 
+/* Device check of the bounded waits: one CTA runs the pipelines' bounded wait on a barrier phase
+ * that nothing completes (role 0, the current limit) and on the phase role 0 would have released
+ * (role 1, four times the limit). On a working device role 0 gives up after the limit, sets
+ * LC_MOE_DEV_WAIT_TIMEOUT in the status word of `ws` and raises the CTA's abort flag, which ends
+ * role 1's wait; the kernel takes about one limit of device time (the default limit is 2 s, so
+ * set a short one with lc_moe_set_wait_limit_ns first) and the context stays usable.
+ * lc_moe_read_status then returns LC_MOE_ERR_TIMEOUT. ws: status only (LC_MOE_OP_STATUS bytes). */
+int lc_moe_check_wait_timeout(void* ws, size_t ws_bytes, void* stream);
+
 /*
  * lc_moe_forward -- the whole MoE layer (MoE equation, section 2.1).
  *   x      [T, d]   bf16   token activations x_t

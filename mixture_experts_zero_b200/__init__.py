@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401,E402
     LcMoeError,
     Shape,
     lc_moe_bias_update,
+    lc_moe_check_wait_timeout,
     lc_moe_combine,
     lc_moe_expert_ffn,
     lc_moe_expert_hist,

@@ -31,6 +31,7 @@ EXPORTED = (
     "lc_moe_read_status", "lc_moe_router_logits", "lc_moe_topk", "lc_moe_expert_hist",
     "lc_moe_permute", "lc_moe_expert_ffn", "lc_moe_combine", "lc_moe_permute_noalloc",
     "lc_moe_quantize_e4m3", "lc_moe_forward_fp8", "lc_moe_forward_fp8_timed",
+    "lc_moe_check_wait_timeout",
 )
 
 
@@ -89,6 +90,7 @@ def _configure(L: ctypes.CDLL) -> ctypes.CDLL:
     fwd8 = [SP, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
     L.lc_moe_forward_fp8.argtypes = fwd8
     L.lc_moe_forward_fp8_timed.argtypes = fwd8 + [ctypes.POINTER(P)]
+    L.lc_moe_check_wait_timeout.argtypes = [P, SZ, P]
     return L
 
 
@@ -289,6 +291,16 @@ def lc_moe_bias_update(bias, counts, T_all: int, N: int, Z: int, K: int, K_e: in
                                      ctypes.c_float(mu), int(bool(reset_counts)), _stream(stream)),
            "lc_moe_bias_update")
     return bias
+
+
+def lc_moe_check_wait_timeout(ws=None, stream=None):
+    """Enqueue the device check of the bounded waits (gives up after the current wait limit and
+    sets LC_MOE_DEV_WAIT_TIMEOUT in ws's status word). Returns the workspace."""
+    if ws is None:
+        ws = new_workspace(Shape(1, 64, 1, 0, 1, 64), OP_STATUS)
+    _check(_lib().lc_moe_check_wait_timeout(_ptr(ws), ws.numel(), _stream(stream)),
+           "lc_moe_check_wait_timeout")
+    return ws
 
 
 def lc_moe_read_status(ws, stream=None, raise_on_error: bool = True) -> int:

@@ -244,6 +244,15 @@ void lc_moe_set_wait_limit_ns(uint64_t limit_ns) {
     g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
 }
 
+int lc_moe_check_wait_timeout(void* ws, size_t ws_bytes, void* stream) {
+    if (!ws) return LC_MOE_ERR_INVALID_ARG;
+    if (ws_bytes < kStatusBytes) return LC_MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(ws)) return LC_MOE_ERR_MISALIGNED;
+    LC_TRY(device_ok());
+    LC_CUDA(launch_wait_check(at<uint32_t>(ws, 0), wait_limit_ns(), static_cast<cudaStream_t>(stream)));
+    return LC_MOE_OK;
+}
+
 int lc_moe_forward(const lc_moe_shape* s, const void* x, const void* wr, const float* bias,
                    const void* w13, const void* w2, void* out, int32_t* idx, float* gate,
                    int32_t* counts, void* ws, size_t ws_bytes, void* stream) {

@@ -409,4 +409,6 @@ cudaError_t launch_combine(const void* x, const void* y, const float* gate,
                            const int32_t* pair_row, int T, int d, int K, void* out,
                            cudaStream_t st);
 
+cudaError_t launch_wait_check(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
+
 }  // namespace lcmoe

@@ -99,6 +99,9 @@ def test_argument_checks_precede_any_cuda_call(lib):
     assert lib.lc_moe_bias_update(p, p, 64, 8, 4, 3, 2, ctypes.c_float(float("nan")), 0, None) == binding.ERR_INVALID_ARG
     assert lib.lc_moe_expert_hist(p, 10, 0, p, p, 256, None) == binding.ERR_INVALID_ARG
     assert lib.lc_moe_read_status(None, None, None) == binding.ERR_INVALID_ARG
+    assert lib.lc_moe_check_wait_timeout(None, 256, None) == binding.ERR_INVALID_ARG
+    assert lib.lc_moe_check_wait_timeout(p, 255, None) == binding.ERR_WORKSPACE_TOO_SMALL
+    assert lib.lc_moe_check_wait_timeout(q, 256, None) == binding.ERR_MISALIGNED
 
 
 def test_valid_call_without_a_device_reports_a_cuda_error(lib):
@@ -109,6 +112,7 @@ def test_valid_call_without_a_device_reports_a_cuda_error(lib):
     p = ctypes.c_void_p(256)
     need = lib.lc_moe_workspace_bytes(ctypes.byref(s), 0)
     assert lib.lc_moe_forward(ctypes.byref(s), p, p, p, p, p, p, None, None, None, p, need, None) == binding.ERR_CUDA
+    assert lib.lc_moe_check_wait_timeout(p, 256, None) == binding.ERR_CUDA
 
 
 def test_the_cuda_package_never_imports_the_oracle():
