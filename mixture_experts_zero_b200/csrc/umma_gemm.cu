@@ -283,12 +283,29 @@ cudaError_t launch_router_gemm(const void* x, const void* wr, float* logits, int
                                uint32_t* status, cudaStream_t st) {
     const DevInfo* di = current_device_info();
     if (!di) return cudaErrorUnknown;
-    int bn = ((E + 31) / 32) * 32;
-    if (bn > 256) bn = 256;
-    // few token tiles (decode-sized T): narrower expert tiles, down to 32, so that more SMs
-    // stream the router weight
+    const int bn_max = ((E + 31) / 32) * 32 < 256 ? ((E + 31) / 32) * 32 : 256;
+    int bn = bn_max;
     const int m_tiles = (T + BM - 1) / BM;
-    while (bn > 32 && m_tiles * ((E + bn - 1) / bn) < di->sm_count) bn = ((bn / 2 + 31) / 32) * 32;
+    const int sms = di->sm_count;
+    if (m_tiles * ((E + bn - 1) / bn) < sms) {
+        // few token tiles (decode-sized T): narrower expert tiles, down to 32, so that more SMs
+        // stream the router weight
+        while (bn > 32 && m_tiles * ((E + bn - 1) / bn) < sms) bn = ((bn / 2 + 31) / 32) * 32;
+    } else {
+        // at least one full wave: the width from bn_max down to 128 (multiples of 32) with the
+        // least waves x width, i.e. the last wave filled best (a tile's time grows with its width);
+        // ties keep the wider tile
+        int64_t best = -1;
+        for (int c = bn_max; c >= 128 || c == bn_max; c -= 32) {
+            const int64_t tiles = static_cast<int64_t>(m_tiles) * ((E + c - 1) / c);
+            const int64_t cost = ((tiles + sms - 1) / sms) * c;
+            if (best < 0 || cost < best) {
+                best = cost;
+                bn = c;
+            }
+            if (c <= 32) break;
+        }
+    }
     CUtensorMap ma, mb;
     if (!make_tma_map_2d(&ma, x, static_cast<uint64_t>(T), d, BM)) return cudaErrorInvalidValue;
     if (!make_tma_map_2d(&mb, wr, static_cast<uint64_t>(E), d, bn)) return cudaErrorInvalidValue;

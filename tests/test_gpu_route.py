@@ -130,7 +130,8 @@ def test_nan_logits_set_the_device_status(cuda_device):
 # tile and of 32 (the top-K kernel's lane stride), ragged token counts past a 128-row M tile,
 # K = 1 and K = 16, with frequent exact ties (small d, integer-grid inputs)
 ROUTE_SHAPES = [(64, 128, 12, 3), (257, 64, 96, 6), (1, 64, 300, 12), (300, 128, 512, 16),
-                (513, 64, 700, 12), (1000, 256, 768, 12), (129, 64, 768, 1), (70, 64, 33, 16)]
+                (513, 64, 700, 12), (1000, 256, 768, 12), (129, 64, 768, 1), (70, 64, 33, 16),
+                (8192, 64, 768, 12), (5000, 64, 2000, 8)]  # the last two: 192-column router tiles
 
 
 @pytest.mark.parametrize("shape", ROUTE_SHAPES, ids=[str(s) for s in ROUTE_SHAPES])
