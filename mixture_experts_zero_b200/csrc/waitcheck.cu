@@ -1,10 +1,11 @@
 // waitcheck.cu -- a device check of the bounded pipeline waits.
 //
-// Every mbarrier wait in the GEMMs and the row gather gives up after a time limit, raises its
-// CTA's abort flag and records LC_MOE_DEV_WAIT_TIMEOUT, so that a stalled pipeline ends as a
-// status the host reads instead of a hung context. This kernel runs that same wait (mbar_wait of
-// common.cuh) on a two-role pipeline whose first phase never completes, so a caller can see on
-// its own device that the limit ends the wait and that the abort reaches the other role:
+// Every mbarrier wait in the GEMMs and the row gather gives up after a time limit and records
+// LC_MOE_DEV_WAIT_TIMEOUT (in the GEMMs the wait also raises its CTA's abort flag, which ends the
+// other roles' waits), so that a stalled pipeline ends as a status the host reads instead of a
+// hung context. This kernel runs the GEMMs' wait (mbar_wait of common.cuh) on a two-role pipeline
+// whose first phase never completes, so a caller can see on its own device that the limit ends
+// the wait and that the abort reaches the other role:
 //   - role 0 waits for phase 0 of `first`, on which nothing ever arrives, with the limit; it
 //     gives up, raises the abort flag and records WAIT_TIMEOUT. (Had it completed, it would have
 //     arrived on `second`.)
