@@ -6,10 +6,10 @@
 // hung context. This kernel runs the GEMMs' wait (mbar_wait of common.cuh) on a two-role pipeline
 // whose first phase never completes, so a caller can see on its own device that the limit ends
 // the wait and that the abort reaches the other role:
-//   - role 0 waits for phase 0 of `first`, on which nothing ever arrives, with the limit; it
+//   - role 0 waits for phase 0 of bars[0], on which nothing ever arrives, with the limit; it
 //     gives up, raises the abort flag and records WAIT_TIMEOUT. (Had it completed, it would have
-//     arrived on `second`.)
-//   - role 1 waits for phase 0 of `second` with four times the limit, and leaves through the
+//     arrived on bars[1].)
+//   - role 1 waits for phase 0 of bars[1] with four times the limit, and leaves through the
 //     abort flag role 0 raised, after about one limit rather than four.
 // Both waits are bounded by their own clocks, so the kernel ends within four limits whatever
 // happens.
