@@ -9,6 +9,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/lc_moe.h"
 
 namespace lcmoe {
@@ -333,6 +336,33 @@ struct DevInfo {
     int sm_count;
     int ok_sm100;
 };
+
+// Host-side set-up that must run once per device before a kernel's first launch there (kernel
+// attributes, symbol addresses). run() calls `fn` on the current device until one call succeeds:
+// concurrent first callers on any host thread are serialised by the mutex and later callers see
+// the release-stored flag without locking; a failed attempt is returned to its caller and tried
+// again by the next call instead of being remembered.
+class PerDeviceOnce {
+  public:
+    static constexpr int kMaxDevices = 64;
+    template <class F>
+    cudaError_t run(F&& fn) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        if (done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        std::lock_guard<std::mutex> lock(mu_);
+        if (done_[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+        e = fn(dev);
+        if (e == cudaSuccess) done_[dev].store(true, std::memory_order_release);
+        return e;
+    }
+
+  private:
+    std::mutex mu_;
+    std::atomic<bool> done_[kMaxDevices] = {};
+};
 // Per-device cached properties of the current device (returns nullptr on a CUDA error).
 const DevInfo* current_device_info();
 
@@ -410,5 +440,12 @@ cudaError_t launch_combine(const void* x, const void* y, const float* gate,
                            cudaStream_t st);
 
 cudaError_t launch_wait_check(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
+
+// Expert parallelism: expert-major permutation of rows received source-major (cnt [G, n_local],
+// G * n_local <= 2048), and a row copy through an index map (gather or scatter).
+cudaError_t launch_regroup_plan(const int32_t* cnt, int G, int n_local, int32_t* perm, int64_t m_cap,
+                                int32_t* offsets, uint32_t* status, cudaStream_t st);
+cudaError_t launch_copy_rows(const void* src, void* dst, const int32_t* map, int64_t n, int row_bytes,
+                             int scatter, uint32_t* status, cudaStream_t st);
 
 }  // namespace lcmoe

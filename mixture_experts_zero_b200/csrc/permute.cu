@@ -283,16 +283,12 @@ cudaError_t launch_gather_rows(const void* x, int T, uint32_t row_bytes, int K, 
     if (T == 0) return cudaSuccess;
     if (row_bytes <= GB_MAX_ROW_BYTES) {
         const size_t smem = static_cast<size_t>(2 * GB_WARPS) * row_bytes;
-        static int configured[64] = {0};
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
+        static PerDeviceOnce setup;
+        const cudaError_t e = setup.run([](int) {
+            return cudaFuncSetAttribute(gather_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(2 * GB_WARPS * GB_MAX_ROW_BYTES));
+        });
         if (e != cudaSuccess) return e;
-        if (dev < 64 && !configured[dev]) {
-            e = cudaFuncSetAttribute(gather_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(2 * GB_WARPS * GB_MAX_ROW_BYTES));
-            if (e != cudaSuccess) return e;
-            configured[dev] = 1;
-        }
         int blocks = (T + GB_WARPS - 1) / GB_WARPS;
         const int per_sm = smem ? static_cast<int>((200u * 1024u) / smem) : 8;
         const int cap = di->sm_count * (per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm));
@@ -324,18 +320,16 @@ cudaError_t launch_permute(const int32_t* idx, int T, int K, int N, int E, int32
     int32_t* cnt = scratch;
     int32_t* base = scratch + static_cast<size_t>(nblk) * N;
     const size_t mask_bytes = static_cast<size_t>(N) * MASK_WORDS * sizeof(uint32_t);
-    static bool configured[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 64 && !configured[dev]) {
+    static PerDeviceOnce setup;
+    cudaError_t e = setup.run([](int) {
         // masks of up to 2048 experts take 64 KB of shared memory
-        e = cudaFuncSetAttribute(perm_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2048 * MASK_WORDS * 4);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(perm_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2048 * MASK_WORDS * 4);
-        if (e != cudaSuccess) return e;
-        configured[dev] = true;
-    }
+        cudaError_t r = cudaFuncSetAttribute(perm_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             2048 * MASK_WORDS * 4);
+        if (r != cudaSuccess) return r;
+        return cudaFuncSetAttribute(perm_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    2048 * MASK_WORDS * 4);
+    });
+    if (e != cudaSuccess) return e;
     if (nblk > 0) {
         perm_count_kernel<<<nblk, PB, mask_bytes, st>>>(idx, T, K, N, E, cnt, status);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -376,22 +370,22 @@ namespace {
 constexpr int64_t kNoAllocTableEntries = 131072;  // per table: 512 KB of int32
 __device__ __align__(256) int32_t g_noalloc_tables[2 * kNoAllocTableEntries];
 
-// Device address of g_noalloc_tables on the current device, looked up once per device. In host
-// code the symbol is only a stand-in for the device array; kernels must get this address.
+// Device address of g_noalloc_tables on the current device. In host code the symbol is only a
+// stand-in for the device array; kernels must get this address. The lookup runs on a device's
+// first call and is kept once it succeeds; a failed lookup (for example one attempted inside a
+// stream capture) is returned and tried again on the next call.
 cudaError_t noalloc_tables_ptr(int32_t** out) {
-    static int32_t* ptrs[64];
-    static cudaError_t errs[64];
-    static std::once_flag flags[64];
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    std::call_once(flags[dev], [dev] {
+    static PerDeviceOnce lookup;
+    static int32_t* ptrs[PerDeviceOnce::kMaxDevices];
+    cudaError_t e = lookup.run([](int dev) {
         void* p = nullptr;
-        errs[dev] = cudaGetSymbolAddress(&p, g_noalloc_tables);
-        ptrs[dev] = static_cast<int32_t*>(p);
+        const cudaError_t r = cudaGetSymbolAddress(&p, g_noalloc_tables);
+        if (r == cudaSuccess) ptrs[dev] = static_cast<int32_t*>(p);
+        return r;
     });
-    if (errs[dev] != cudaSuccess) return errs[dev];
+    if (e != cudaSuccess) return e;
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     *out = ptrs[dev];
     return cudaSuccess;
 }

@@ -322,16 +322,12 @@ cudaError_t launch_router_gemm(const void* x, const void* wr, float* logits, int
     const int tiles = ((T + BM - 1) / BM) * a.ntiles;
     const int grid = tiles < di->sm_count ? tiles : di->sm_count;
     const size_t smem = SmemLayout::bytes();
-    static bool configured[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static PerDeviceOnce setup;
+    const cudaError_t e = setup.run([smem](int) {
+        return cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(smem));
+    });
     if (e != cudaSuccess) return e;
-    if (dev < 64 && !configured[dev]) {
-        e = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        configured[dev] = true;
-    }
     router_gemm_kernel<<<grid, NUM_THREADS, smem, st>>>(ma, mb, a);
     return cudaGetLastError();
 }

@@ -1,11 +1,13 @@
-"""The allocation-free grouping entry point, lc_moe_permute_noalloc, against lc_moe_permute.
+"""The allocation-free grouping entry point, lc_moe_permute_noalloc, against lc_moe_permute and
+against the CPU oracle's grouping.
 
 Some callers cannot allocate device memory: an engine whose memory planner hands out all device
 memory up front and refuses later requests, or a caller with no workspace of its own to pass.
 For them lc_moe_permute_noalloc keeps the grouping tables in a fixed-size array inside the
 library. Its results must equal lc_moe_permute's bit for bit (integer tables and row copies are
 exact), on two calls in a row with different shapes, so the second call cannot depend on what the
-first one left in the shared array.
+first one left in the shared array. Its integer tables must also equal the oracle's grouping
+(FFN picks ordered by expert, then by token), which shares no code with either GPU path.
 """
 import ctypes
 
@@ -13,6 +15,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from mixture_experts_zero_b200 import binding as B
 from mixture_experts_zero_b200 import inputs
 
@@ -47,6 +50,14 @@ def test_noalloc_grouping_equals_workspace_grouping_on_two_calls(cuda_device):
         assert torch.equal(got[3][:M], want[3][:M])            # grouped rows
         assert int(status.item()) == 0
         assert 0 < M < idx.numel()
+        # the oracle's grouping of the same picks: offsets, row -> token, pick -> row
+        o_off, o_row_token, o_pair_row = oracle.permute(idx.cpu().numpy(), N)
+        assert np.array_equal(got[0].cpu().numpy(), o_off)
+        assert np.array_equal(got[1][:M].cpu().numpy(), o_row_token)
+        assert np.array_equal(got[2].cpu().numpy(), o_pair_row)
+        # grouped rows are the token rows named by the oracle's row -> token table
+        xb = inputs.bits(x)
+        assert np.array_equal(inputs.bits(got[3][:M]), xb[o_row_token])
 
 
 def test_noalloc_grouping_rejects_shapes_beyond_its_capacity(cuda_device):
