@@ -393,7 +393,8 @@ def run_ours(args):
         "clocks": ClockSampler.summarize(clock_rows),
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline and not f8:
-        result["cpu_baseline"] = cpu_baseline(w, data, budget_s=args.cpu_budget)
+        result["cpu_baseline"] = cpu_baseline(w, data, route_tokens=args.cpu_route_tokens,
+                                              ffn_tokens=args.cpu_ffn_tokens)
     if world > 1:
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
@@ -403,67 +404,111 @@ def run_ours(args):
 
 # ------------------------------------------------------------------- oracle (CPU baseline) ---
 
-def oracle_sample_step(w, x_bits, wr_bits, bias, expert_fetch, tokens):
-    """Run the oracle on ``tokens`` of the batch; return (seconds of oracle compute, n tokens)."""
+def _ffn_pairs(idx, tokens, N):
+    """FFN picks (token, rank) of ``tokens`` under routing idx, and their experts."""
+    pairs = [(int(t), r) for t in tokens for r in range(idx.shape[1]) if idx[t, r] < N]
+    experts = np.array([idx[t, r] for t, r in pairs], np.int64)
+    return pairs, experts
+
+
+def _oracle_ffn(w, x_bits, pairs, experts, expert_weights, chunk: int):
+    """Oracle SwiGLU rows of every FFN pick in ``pairs``, one ``oracle.expert_rows`` call per group
+    of ``chunk`` distinct experts (every row of those experts in one call, so the oracle's OpenMP
+    loop over rows has many rows to spread). ``expert_weights(list)`` returns host copies
+    (w13 [n, 2I, d], w2 [n, d, I]) of the listed experts; it runs outside the timed calls.
+    Returns (Y [len(pairs), d], seconds inside the oracle, rows per call)."""
     import oracle
-    t0 = time.perf_counter()
-    xs = np.ascontiguousarray(x_bits[tokens])
-    z = oracle.router_logits(xs, wr_bits)
-    idx, gate, _, _ = oracle.route(z, bias, w.K)
-    t_oracle = time.perf_counter() - t0
-    pairs = [(i, r) for i in range(len(tokens)) for r in range(w.K) if idx[i, r] < w.N]
     Y = np.empty((len(pairs), w.d), np.uint16)
-    pr = np.full((len(tokens), w.K), -1, np.int32)
-    experts = np.array([idx[i, r] for i, r in pairs], np.int64)
-    for e in np.unique(experts):
-        sel = np.nonzero(experts == e)[0]
-        w13e, w2e = expert_fetch(int(e))           # host copy, not timed
-        rows = np.ascontiguousarray(xs[[pairs[j][0] for j in sel]])
+    uniq = np.unique(experts)
+    t_oracle = 0.0
+    rows_per_call = []
+    for c0 in range(0, uniq.size, chunk):
+        group = uniq[c0:c0 + chunk]
+        w13c, w2c = expert_weights(group.tolist())
+        local = {int(e): i for i, e in enumerate(group)}
+        sel = np.nonzero(np.isin(experts, group))[0]
+        rows = np.ascontiguousarray(x_bits[[pairs[j][0] for j in sel]])
+        row_expert = np.array([local[int(experts[j])] for j in sel], np.int32)
         t0 = time.perf_counter()
-        _, y = oracle.expert_rows(rows, np.zeros(sel.size, np.int32), w13e, w2e, want_h=False)
+        _, y = oracle.expert_rows(rows, row_expert, w13c, w2c, want_h=False)
         t_oracle += time.perf_counter() - t0
         Y[sel] = y
-    for j, (i, r) in enumerate(pairs):
-        pr[i, r] = j
+        rows_per_call.append(int(sel.size))
+    return Y, t_oracle, rows_per_call
+
+
+def _oracle_combine(w, x_bits, tokens, idx, gate, pairs, Y):
+    import oracle
+    pos = {int(t): i for i, t in enumerate(tokens)}
+    pr = np.full((len(tokens), w.K), -1, np.int32)
+    for j, (t, r) in enumerate(pairs):
+        pr[pos[t], r] = j
+    xs = np.ascontiguousarray(x_bits[tokens])
     t0 = time.perf_counter()
-    oracle.combine(xs, Y, idx, gate, pr, w.N)
-    t_oracle += time.perf_counter() - t0
-    return t_oracle, len(tokens)
+    oracle.combine(xs, Y, np.ascontiguousarray(idx[tokens]), np.ascontiguousarray(gate[tokens]), pr, w.N)
+    return time.perf_counter() - t0
 
 
-def cpu_baseline(w, data, budget_s: float = 20.0):
+def cpu_baseline(w, data, route_tokens: int | None = None, ffn_tokens: int = 256, chunk: int = 64):
+    """The oracle on the host cores, on a bounded sample of the batch, in three timed phases:
+    routing (router logits, softmax, biased top-K) of the first ``route_tokens`` tokens (all T by
+    default); the SwiGLU experts of every FFN pick of a seeded subset of ``ffn_tokens`` of them,
+    batched per group of ``chunk`` experts (the weights of each group copied to the host outside
+    the timed calls); and the combine of that subset. tokens/s = 1 / (routing s per token +
+    expert and combine s per token), each per-token cost measured on its own sample."""
     import oracle
     from mixture_experts_zero_b200 import inputs
-    x_bits = inputs.bits(data["x"])
+    R = w.T if route_tokens is None else min(route_tokens, w.T)
+    x_bits = inputs.bits(data["x"])[:R]
     wr_bits = inputs.bits(data["wr"])
     bias = data["bias"].cpu().numpy()
-
-    def fetch(e):
-        return (inputs.bits(data["w13"][e]).reshape(1, 2 * w.I, w.d),
-                inputs.bits(data["w2"][e]).reshape(1, w.d, w.I))
-
+    t0 = time.perf_counter()
+    z = oracle.router_logits(x_bits, wr_bits)
+    idx, gate, _, _ = oracle.route(z, bias, w.K)
+    t_route = time.perf_counter() - t0
+    del z
     rng = np.random.default_rng(123)
-    n = 4
-    spent = tok = 0.0
-    while spent < budget_s:
-        tokens = np.sort(rng.choice(w.T, n, replace=False))
-        s, k = oracle_sample_step(w, x_bits, wr_bits, bias, fetch, tokens)
-        spent += s
-        tok += k
-        if spent < budget_s / 4:
-            n = min(n * 2, 64)
-    return {"value": round(tok / spent, 3), "unit": UNIT, "cores": oracle.num_threads(),
-            "cpu": cpu_model(), "host_cpus": os.cpu_count(),
-            "kind": "oracle",
-            "sample": f"{int(tok)} random tokens of the {w.name} batch (router logits, routing, "
-                      f"SwiGLU experts of their FFN picks, combine), {spent:.1f} s of oracle time; "
-                      "expert weights copied to the host per expert outside the timed calls"}
+    F = min(ffn_tokens, R)
+    tokens = np.sort(rng.choice(R, F, replace=False))
+    pairs, experts = _ffn_pairs(idx, tokens, w.N)
+    w13h = np.empty((chunk, 2 * w.I, w.d), np.uint16)
+    w2h = np.empty((chunk, w.d, w.I), np.uint16)
+
+    def weights(group):
+        for i, e in enumerate(group):
+            w13h[i] = inputs.bits(data["w13"][e])
+            w2h[i] = inputs.bits(data["w2"][e])
+        return w13h[:len(group)], w2h[:len(group)]
+
+    Y, t_ffn, rows_per_call = _oracle_ffn(w, x_bits, pairs, experts, weights, chunk)
+    t_comb = _oracle_combine(w, x_bits, tokens, idx, gate, pairs, Y)
+    value = 1.0 / (t_route / R + (t_ffn + t_comb) / F)
+    threads = oracle.num_threads()
+    return {"value": round(value, 3), "unit": UNIT, "cores": threads,
+            "cpu": cpu_model(), "host_cpus": os.cpu_count(), "kind": "oracle",
+            "sample": (f"subset-measured: routing of {R} tokens of the {w.name} batch "
+                       f"({t_route:.2f} s), SwiGLU experts of the {len(pairs)} FFN picks of {F} "
+                       f"seeded tokens of them ({t_ffn:.2f} s, {len(rows_per_call)} oracle calls "
+                       f"of {min(rows_per_call)}-{max(rows_per_call)} rows, every row of up to "
+                       f"{chunk} experts per call) and their combine ({t_comb:.3f} s); every "
+                       f"phase runs the oracle's OpenMP loops on {threads} threads; the GPU arm's "
+                       f"expert weights, copied to the host outside the timed calls"),
+            "phases_s": {"route": round(t_route, 3), "experts": round(t_ffn, 3),
+                         "combine": round(t_comb, 4)},
+            "tokens": {"routed": R, "ffn": F, "ffn_picks": len(pairs)}}
 
 
 # --------------------------------------------------------------------------- reference arm --
 
+REF_WEIGHT_SETS = 16
+
+
 def run_reference(args):
-    """The oracle (CPU, plain C) as the reference arm, on bounded samples of the same workload."""
+    """The oracle (CPU, plain C) as the reference arm, on bounded samples of the same workload:
+    each step routes ``--ref-tokens`` fresh tokens and runs every FFN pick of them through the
+    SwiGLU experts (one oracle call for all of a step's picks) and the combine. Expert weights
+    are drawn on the host: expert e uses weight set e mod 16 of 16 seeded sets (the oracle's cost
+    does not depend on the values; the GPU arm's 38.6 GB of weights are not copied)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -474,40 +519,57 @@ def run_reference(args):
     g = inputs.generator(w.seed, "cpu")
     wr_bits = inputs.bits(inputs.draw_router(w, g, "cpu"))
     bias = inputs.draw_bias(w, g, "cpu").numpy()
-    cache = {}
     std = 1.0 / math.sqrt(w.d)
-
-    def fetch(e):
-        if e not in cache:
-            ge = inputs.generator(w.seed * 100003 + e, "cpu")
-            w13 = (torch.randn(1, 2 * w.I, w.d, generator=ge) * std).to(torch.bfloat16)
-            w2 = (torch.randn(1, w.d, w.I, generator=ge) * std).to(torch.bfloat16)
-            cache[e] = (inputs.bits(w13), inputs.bits(w2))
-        return cache[e]
+    P = min(REF_WEIGHT_SETS, w.N)
+    ge = inputs.generator(w.seed * 100003, "cpu")
+    w13s = inputs.bits((torch.randn(P, 2 * w.I, w.d, generator=ge) * std).to(torch.bfloat16))
+    w2s = inputs.bits((torch.randn(P, w.d, w.I, generator=ge) * std).to(torch.bfloat16))
 
     per_step_tokens = args.ref_tokens
-    total_s = total_tok = 0.0
+    total = {"route": 0.0, "experts": 0.0, "combine": 0.0}
+    picks = 0
     for i in range(args.warmup + args.steps):
         gx = inputs.generator(w.seed * 7919 + i, "cpu")
         xs = torch.randn(per_step_tokens, w.d, generator=gx)
         if w.router == "zipf":
             xs[:, 0] = 1.0
         x_bits = inputs.bits(xs.to(torch.bfloat16))
-        s, k = oracle_sample_step(w, x_bits, wr_bits, bias, fetch, np.arange(per_step_tokens))
+        t0 = time.perf_counter()
+        z = oracle.router_logits(x_bits, wr_bits)
+        idx, gate, _, _ = oracle.route(z, bias, w.K)
+        t_route = time.perf_counter() - t0
+        tokens = np.arange(per_step_tokens)
+        pairs, experts = _ffn_pairs(idx, tokens, w.N)
+        Y, t_ffn, _ = _oracle_ffn(w, x_bits, pairs, experts % P,
+                                  lambda group: (w13s[group], w2s[group]), P)
+        t_comb = _oracle_combine(w, x_bits, tokens, idx, gate, pairs, Y)
         if i >= args.warmup:
-            total_s += s
-            total_tok += k
-    value = total_tok / total_s
+            total["route"] += t_route
+            total["experts"] += t_ffn
+            total["combine"] += t_comb
+            picks += len(pairs)
+    total_s = sum(total.values())
+    value = per_step_tokens * args.steps / total_s
+    config = workload_config(w, int(os.environ.get("WORLD_SIZE", "1")), False)
+    config.update({"T_sampled": per_step_tokens,
+                   "sample": f"{per_step_tokens} fresh tokens per step (not the T={w.T} batch)",
+                   "expert_weights": f"drawn on the host: expert e uses set e mod {P} of {P} "
+                                     "seeded sets, not the GPU arm's weights"})
+    threads = oracle.num_threads()
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_s / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, int(os.environ.get("WORLD_SIZE", "1")), False),
-        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.num_threads(),
+        "config": config,
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": threads,
                          "cpu": cpu_model(), "host_cpus": os.cpu_count(),
                          "kind": "oracle",
-                         "sample": f"{per_step_tokens} fresh tokens per step of the {w.name} workload"},
+                         "sample": (f"{per_step_tokens} fresh tokens per step of the {w.name} "
+                                    f"workload: routing, their {picks} FFN picks over the timed "
+                                    f"steps (one oracle call per step), combine; the oracle's "
+                                    f"OpenMP loops on {threads} threads"),
+                         "phases_s": {k: round(v, 3) for k, v in total.items()}},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
@@ -665,8 +727,11 @@ def main():
     ap.add_argument("--workload", default="prefill",
                     choices=["prefill", "decode", "small", "tiny", "prefill_ncu", "route_ncu"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time")
-    ap.add_argument("--ref-tokens", type=int, default=4, help="tokens per reference-arm step")
+    ap.add_argument("--cpu-route-tokens", type=int, default=None,
+                    help="tokens the CPU baseline routes (default: the whole batch)")
+    ap.add_argument("--cpu-ffn-tokens", type=int, default=256,
+                    help="tokens whose FFN picks the CPU baseline runs through the experts")
+    ap.add_argument("--ref-tokens", type=int, default=8, help="tokens per reference-arm step")
     ap.add_argument("--experts", choices=["bf16", "fp8"], default="bf16",
                     help="fp8: E4M3 expert projections (lc_moe_forward_fp8)")
     ap.add_argument("--sweep", choices=["ffn_rows", "hist", "control"], default=None,

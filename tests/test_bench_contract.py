@@ -31,8 +31,12 @@ def test_reference_arm_prints_one_json_line_with_the_contract_keys():
     assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
     assert d["steps"] == 3 and d["warmup"] == 3 and d["n_gpus"] == 1
     assert d["config"]["workload"].startswith("tiny")
+    # the line states what each step ran: a few fresh tokens, host-drawn weights
+    assert d["config"]["T_sampled"] == 8 and "fresh tokens per step" in d["config"]["sample"]
+    assert "not the GPU arm's weights" in d["config"]["expert_weights"]
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert set(cb["phases_s"]) == {"route", "experts", "combine"}
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
@@ -49,3 +53,23 @@ def test_fewer_than_three_warmup_steps_are_refused():
     r = run(["--impl", "reference", "--workload", "tiny", "--steps", "3", "--warmup", "2"])
     assert r.returncode != 0
     assert "--warmup must be >= 3" in r.stderr
+
+
+def test_cpu_baseline_batches_the_expert_rows_and_names_its_phases():
+    """The GPU arm's CPU baseline, run here on the tiny workload's host tensors: every FFN pick of
+    the sampled tokens goes through the oracle in calls of many rows (grouped by expert), and the
+    line names the routed and FFN token counts, the per-phase times and the thread count."""
+    sys.path.insert(0, str(ROOT))
+    import bench
+    import oracle
+    from mixture_experts_zero_b200 import inputs
+    w = inputs.WORKLOADS["tiny"]
+    data = inputs.make(w, device="cpu")
+    cb = bench.cpu_baseline(w, data, ffn_tokens=32, chunk=4)
+    assert cb["value"] > 0 and cb["kind"] == "oracle"
+    assert cb["cores"] == oracle.num_threads()
+    assert cb["tokens"]["routed"] == w.T and cb["tokens"]["ffn"] == 32
+    assert cb["tokens"]["ffn_picks"] > 0
+    assert "subset-measured" in cb["sample"] and f"{cb['cores']} threads" in cb["sample"]
+    # N = 8 experts in groups of 4: two oracle calls, each with the rows of four experts
+    assert "2 oracle calls" in cb["sample"]
