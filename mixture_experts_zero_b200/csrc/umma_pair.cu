@@ -11,23 +11,32 @@
 // Per SM this halves the B bytes loaded per FLOP compared with a 128-row tile, which lowers the
 // L2-to-SM traffic of the main loop by a third.
 //
-// Roles (256 threads per CTA):
+// Roles (384 threads per CTA):
 //   warp 0, one lane, both CTAs  TMA producer: loads this CTA's share of each stage; the bytes
 //                                 complete on the leader's full barrier, where the leader alone
 //                                 posts the expected byte count of the pair;
 //   warp 1, one lane, leader     MMA issuer; tcgen05.commit with a 2-CTA multicast releases the
 //                                 stage in both CTAs and publishes finished accumulators to both;
 //   warp 1, both CTAs            TMEM allocation / deallocation (512 columns, cta_group::2);
-//   warps 4..7, both CTAs        epilogue of this CTA's 128 accumulator lanes; each warp arrives
-//                                 on the leader's accumulator-empty barrier (8 arrivals).
+//   warps 4..11, both CTAs       two epilogue groups of four warps; group g drains accumulator g
+//                                 (TMEM columns [256 g, 256 g + 256)) over this CTA's 128 lanes,
+//                                 and each of its warps arrives on the leader's accumulator-empty
+//                                 barrier g (8 arrivals: 4 warps in each CTA).
 //
 // Tile kinds:
 //   row tiles: 256 rows of one expert. GEMM 1: the leader loads 128 gate rows and its peer the
 //     matching 128 up rows of B, so accumulator columns [0, 128) hold gate and [128, 256) hold up
-//     values for every row. GEMM 2: 256 output features, 128 per CTA.
+//     values for every row. GEMM 2: 256 output features, 128 per CTA. A "wide" row tile (when I is
+//     a multiple of 256 for GEMM 1, d a multiple of 512 for GEMM 2) loads a second box of B rows
+//     one tile width further on and issues a second MMA on the same A into the other accumulator:
+//     256 rows x 512 accumulator columns per tile, so the row operand is read once per 512
+//     columns instead of once per 256, a quarter fewer bytes from L2 per FLOP. Its two halves
+//     are drained by the two epilogue groups in parallel.
 //   weight tiles ("swap"): 256 weight rows (128 per CTA) on the M side and the rows of one expert,
 //     rounded up to 64 and split between the CTAs, on the N side (N <= 128 for GEMM 1, <= 256 for
 //     GEMM 2). GEMM 1 issues a gate MMA into columns [0, N) and an up MMA into [128, 128 + N).
+// Accumulators: a wide row tile takes both; every other tile takes the next one in turn, so the
+// epilogue of one weight tile or narrow row tile overlaps the main loop of the next.
 // Per expert with c_e rows: below cold_rows it is "cold" and runs as weight tiles only; otherwise
 // it runs floor(c_e / 256) row tiles, and its leftover rows run as one more row tile if there are
 // at least rem_rows of them, else as weight tiles (N rounded up to 64). GEMM 1: cold_rows =
@@ -54,7 +63,8 @@ constexpr int A_BYTES = HALF_M * BK * 2;    // 16 KB
 constexpr int B_SLOT = 2 * A_BYTES;         // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_SLOT;
 constexpr int TMEM_COLS = 512;
-constexpr int NUM_THREADS = 256;
+constexpr int NUM_THREADS = 384;
+constexpr int EPI_WARP0 = 4;              // warps 4..11: two epilogue groups of four warps
 constexpr int TOK_BOX = 32;                 // token rows per TMA box of a weight tile (per CTA)
 constexpr int TOK_ROUND = 2 * TOK_BOX;      // weight-tile N is a multiple of this
 
@@ -78,6 +88,7 @@ struct PairArgs {
     int cold_rows;           // experts with 0 < rows < cold_rows use weight tiles only
     int rem_rows;            // an expert's rows past its last full 256-row tile: fewer than this
                              // run as weight tiles, otherwise as one more row tile
+    int wide;                // row tiles span two accumulators (2 * tile_cols output columns)
     const float* row_scale;  // E4M3 GEMM 1: scale of each grouped row [rows_cap]
     const float* w_scale;    // E4M3 GEMM 1: scale of each weight row [n_groups * b_group_rows]
 };
@@ -93,17 +104,32 @@ struct Layout {
     static constexpr int n_bars = 2 * STAGES + 5;  // full, empty, tfull[2], tempty[2], drain
     static constexpr int misc_off = bars_off + n_bars * 8;
     static constexpr int xpose_off = (misc_off + 16 + 127) & ~127;
-    static constexpr int table_off = xpose_off + 4 * XPOSE_WARP;
-    static size_t bytes(int n_groups) { return 1024 + table_off + 3 * static_cast<size_t>(n_groups + 1) * 4; }
+    static constexpr int table_off = xpose_off + 8 * XPOSE_WARP;
+    static size_t bytes(int n_groups) { return 1024 + table_off + 2 * static_cast<size_t>(n_groups + 1) * 4; }
 };
 
 struct Tile {
     int swap;
+    int wide;  // row tile over both accumulators
     int grp;
     int64_t row0;
     int rows;
     int n0;
     int ntok;  // weight tile: MMA N
+};
+
+// Which TMEM accumulators (two of 256 columns) each tile uses, followed identically by the MMA
+// issuer and the two epilogue groups: a wide row tile takes both; every other tile takes the
+// next one in turn. Bit b of `phase` is the parity of buffer b's current use.
+struct AccSchedule {
+    int next = 0;
+    uint32_t phase = 0u;
+    __device__ __forceinline__ int buffers(int wide) const { return wide ? 3 : (1 << next); }
+    __device__ __forceinline__ uint32_t parity(int b) const { return (phase >> b) & 1u; }
+    __device__ __forceinline__ void advance(int wide) {
+        phase ^= static_cast<uint32_t>(buffers(wide));
+        if (!wide) next ^= 1;
+    }
 };
 
 __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
@@ -150,8 +176,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     uint64_t* drain = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Layout::misc_off);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Layout::misc_off + 4);
-    int32_t* offs_s = reinterpret_cast<int32_t*>(smem + Layout::table_off);
-    int32_t* rpre_s = offs_s + (g.n_groups + 1);
+    // group row offsets are read from global memory (L1-resident after the first tiles); shared
+    // memory holds the per-expert tile prefix sums
+    const int32_t* __restrict__ offs = g.offsets;
+    int32_t* rpre_s = reinterpret_cast<int32_t*>(smem + Layout::table_off);
     int32_t* spre_s = rpre_s + (g.n_groups + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -181,7 +209,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         tmem_alloc_pair(tmem_slot, TMEM_COLS);
         tmem_relinquish_pair();
     }
-    for (int e = threadIdx.x; e <= g.n_groups; e += NUM_THREADS) offs_s[e] = g.offsets[e];
     __syncthreads();
     if (warp == 2) {
         // per expert: tiles of the hot part (row tiles + weight tiles of the leftover rows) and
@@ -195,7 +222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const int e = base + lane;
             int nh = 0, nc = 0;
             if (e < g.n_groups) {
-                int cnt = offs_s[e + 1] - offs_s[e];
+                int cnt = __ldg(offs + (e + 1)) - __ldg(offs + (e));
                 if (cnt < 0) {
                     cnt = 0;
                     set_status(g.status, LC_MOE_DEV_IDX_RANGE);
@@ -244,7 +271,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             // hot expert: its row tiles, then weight tiles for the rows past its last row tile
             const int e = upper_group(rpre_s, g.n_groups, tile);
             const int local = tile - rpre_s[e];
-            const int cnt = offs_s[e + 1] - offs_s[e];
+            const int cnt = __ldg(offs + (e + 1)) - __ldg(offs + (e));
             const int nfull = cnt / (2 * HALF_M);
             const int rem = cnt - nfull * 2 * HALF_M;
             const int nrow = (nfull + (rem >= g.rem_rows ? 1 : 0)) * g.ntiles;
@@ -252,13 +279,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             if (local < nrow) {
                 const int mt = local / g.ntiles;
                 tl.swap = 0;
-                tl.row0 = static_cast<int64_t>(offs_s[e]) + static_cast<int64_t>(mt) * 2 * HALF_M;
+                tl.wide = g.wide;
+                tl.row0 = static_cast<int64_t>(__ldg(offs + (e))) + static_cast<int64_t>(mt) * 2 * HALF_M;
                 tl.rows = min(2 * HALF_M, cnt - mt * 2 * HALF_M);
-                tl.n0 = (local - mt * g.ntiles) * g.tile_cols;
+                tl.n0 = (local - mt * g.ntiles) * g.tile_cols * (g.wide ? 2 : 1);
                 tl.ntok = 0;
             } else {
                 tl.swap = 1;
-                tl.row0 = static_cast<int64_t>(offs_s[e]) + static_cast<int64_t>(nfull) * 2 * HALF_M;
+                tl.wide = 0;
+                tl.row0 = static_cast<int64_t>(__ldg(offs + (e))) + static_cast<int64_t>(nfull) * 2 * HALF_M;
                 tl.rows = rem;
                 tl.n0 = (local - nrow) * 2 * HALF_M;
                 tl.ntok = (rem + TOK_ROUND - 1) / TOK_ROUND * TOK_ROUND;
@@ -268,9 +297,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const int idx = tile - total_r;
             const int e = upper_group(spre_s, g.n_groups, idx);
             tl.swap = 1;
+            tl.wide = 0;
             tl.grp = e;
-            tl.row0 = offs_s[e];
-            tl.rows = offs_s[e + 1] - offs_s[e];
+            tl.row0 = __ldg(offs + (e));
+            tl.rows = __ldg(offs + (e + 1)) - __ldg(offs + (e));
             tl.n0 = (idx - spre_s[e]) * 2 * HALF_M;
             tl.ntok = (tl.rows + TOK_ROUND - 1) / TOK_ROUND * TOK_ROUND;
         }
@@ -289,7 +319,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const Tile tl = decode(tile);
             const int tok_rows = tl.ntok / 2;  // this CTA's share of the N side
             uint32_t cta_bytes;
-            if (!tl.swap) cta_bytes = A_BYTES + A_BYTES;
+            if (!tl.swap) cta_bytes = (tl.wide ? 3 : 2) * A_BYTES;
             else cta_bytes = (MODE == MODE_SWIGLU ? 2 : 1) * A_BYTES + tok_rows * BK * 2;
             const int wbase = tl.grp * g.b_group_rows;
             for (int kb = 0; kb < nk; ++kb) {
@@ -308,6 +338,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     const int wrow = (MODE == MODE_SWIGLU) ? wbase + tl.n0 + static_cast<int>(rank) * g.up_off
                                                            : wbase + tl.n0 + static_cast<int>(rank) * HALF_M;
                     tma_load_2d_pair(sb, &mapW, bar, kx, wrow, pol_normal);
+                    // wide tile: the weight rows of the second accumulator (the next tile_cols
+                    // output columns), one box further on
+                    if (tl.wide) tma_load_2d_pair(sb + A_BYTES, &mapW, bar, kx, wrow + g.tile_cols, pol_normal);
                 } else {
                     const int wrow = wbase + tl.n0 + static_cast<int>(rank) * HALF_M;
                     tma_load_2d_pair(sa, &mapW, bar, kx, wrow, pol_stream);
@@ -342,18 +375,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         // ------------------------------------------------------- MMA issuer (leader only) --
         int s = 0;
         uint32_t ph = 0;
-        int acc = 0;
-        uint32_t aph = 0;
+        AccSchedule sched;
         bool ok = true;
         for (int tile = cluster; tile < total && ok; tile += n_clusters) {
             const Tile tl = decode(tile);
             const uint32_t idesc = F8 ? idesc_e4m3_f32(2 * HALF_M, tl.swap ? tl.ntok : 2 * HALF_M)
                                       : idesc_bf16_f32(2 * HALF_M, tl.swap ? tl.ntok : 2 * HALF_M);
-            if (!mbar_wait(&tempty[acc], aph ^ 1u, g.wait_ns, abort_flag, g.status)) {
-                ok = false;
-                break;
-            }
+            const int bufs = sched.buffers(tl.wide);
+            for (int b = 0; b < 2 && ok; ++b)
+                if ((bufs >> b) & 1) ok = mbar_wait(&tempty[b], sched.parity(b) ^ 1u, g.wait_ns, abort_flag, g.status);
+            if (!ok) break;
             tc_fence_after();
+            const int acc = tl.wide ? 0 : sched.next;
             const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
             for (int kb = 0; kb < nk; ++kb) {
                 if (!mbar_wait(&full[s], ph, g.wait_ns, abort_flag, g.status)) {
@@ -371,6 +404,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         mma_step<F8>(d_tmem, ad + 2 * kk, td + 2 * kk, idesc, (kb | kk) != 0);
                         mma_step<F8>(d_tmem + 128, bd + 2 * kk, td + 2 * kk, idesc, (kb | kk) != 0);
                     }
+                } else if (tl.wide) {
+                    // second accumulator: the weight rows one box further on in shared memory
+                    const uint64_t bd2 = sw128_kmajor_desc(smem_u32(sa + 2 * A_BYTES));
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        mma_step<F8>(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                        mma_step<F8>(d_tmem + 256, ad + 2 * kk, bd2 + 2 * kk, idesc, (kb | kk) != 0);
+                    }
                 } else {
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
@@ -383,25 +424,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 }
             }
             if (!ok) break;
-            umma_commit_pair(&tfull[acc], 0x3);
-            acc ^= 1;
-            if (acc == 0) aph ^= 1u;
+            for (int b = 0; b < 2; ++b)
+                if ((bufs >> b) & 1) umma_commit_pair(&tfull[b], 0x3);
+            sched.advance(tl.wide);
         }
         umma_commit_pair(drain, 0x1);
         wait_drain(drain, 0, g.wait_ns);
-    } else if (warp >= 4) {
+    } else if (warp >= EPI_WARP0) {
         // ------------------------------------------------------------ epilogue (both CTAs) --
-        const int q = warp - 4;
-        int acc = 0;
-        uint32_t aph = 0;
+        // group eg drains accumulator eg: its own tiles, or its half of a wide row tile; warp
+        // w may only read TMEM lanes 32 * (w % 4) .. + 31
+        const int q = warp & 3;
+        const int eg = (warp - EPI_WARP0) >> 2;
+        const int acc = eg;
+        AccSchedule sched;
         __nv_bfloat16* out = g.out;
         for (int tile = cluster; tile < total; tile += n_clusters) {
             const Tile tl = decode(tile);
-            if (!mbar_wait(&tfull[acc], aph, g.wait_ns, abort_flag, g.status)) break;
+            if (!((sched.buffers(tl.wide) >> acc) & 1)) {
+                sched.advance(tl.wide);
+                continue;
+            }
+            if (!mbar_wait(&tfull[acc], sched.parity(acc), g.wait_ns, abort_flag, g.status)) break;
             tc_fence_after();
             const uint32_t tb =
                 tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * 256);
             const int i = q * 32 + lane;  // TMEM lane of this thread
+            // first output column of this accumulator (the second half of a wide row tile starts
+            // tile_cols further on)
+            const int fbase = tl.n0 + (tl.wide ? acc * g.tile_cols : 0);
             if (!tl.swap) {
                 const int r = static_cast<int>(rank) * HALF_M + i;  // row within the 256-row tile
                 const int64_t grow = tl.row0 + r;
@@ -412,7 +463,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         tmem_ld_32x32b_x32(tb + c, gv);
                         tmem_ld_32x32b_x32(tb + HALF_M + c, uv);
                         tmem_ld_wait();
-                        const int f0 = tl.n0 + c;
+                        const int f0 = fbase + c;
                         if (valid && f0 < g.n_out) {
                             if (F8) {
                                 // (acc * row scale) * weight-row scale, gate and up separately
@@ -448,7 +499,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         uint32_t v[32];
                         tmem_ld_32x32b_x32(tb + c, v);
                         tmem_ld_wait();
-                        const int f0 = tl.n0 + c;
+                        const int f0 = fbase + c;
                         if (valid && f0 < g.n_out) {
                             if (F8) {
                                 // (acc * row scale) * weight-row scale
@@ -479,7 +530,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 // weight tile: lane = output feature, column = row of the expert's group. Each
                 // 32 x 32 block goes through shared memory transposed, so that every thread then
                 // stores 32 consecutive features of one row as four 16-byte vectors.
-                uint8_t* xp = smem + Layout::xpose_off + q * XPOSE_WARP;
+                uint8_t* xp = smem + Layout::xpose_off + (warp - EPI_WARP0) * XPOSE_WARP;
                 const int f0 = tl.n0 + static_cast<int>(rank) * HALF_M + q * 32;  // warp's first feature
                 for (int c0 = 0; c0 < tl.ntok; c0 += 32) {
                     uint32_t v[32];
@@ -541,8 +592,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
-            acc ^= 1;
-            if (acc == 0) aph ^= 1u;
+            sched.advance(tl.wide);
         }
     }
 
@@ -558,19 +608,21 @@ template <int MODE, bool F8>
 cudaError_t launch_pair(const CUtensorMap& mr, const CUtensorMap& mw, const CUtensorMap& mt,
                         const PairArgs& args, int grid, cudaStream_t st) {
     const size_t smem = Layout::bytes(args.n_groups);
-    static int configured[64] = {0};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    // once per device: allow the kernel the device's whole opt-in shared memory
+    static PerDeviceOnce setup;
+    static int max_optin[PerDeviceOnce::kMaxDevices];
+    cudaError_t e = setup.run([](int dev) {
+        int v = 0;
+        cudaError_t r = cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (r != cudaSuccess) return r;
+        r = cudaFuncSetAttribute(umma_pair_kernel<MODE, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, v);
+        if (r == cudaSuccess) max_optin[dev] = v;
+        return r;
+    });
     if (e != cudaSuccess) return e;
-    if (dev < 64 && configured[dev] < static_cast<int>(smem)) {
-        int max_optin = 0;
-        e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-        if (e != cudaSuccess) return e;
-        if (static_cast<int>(smem) > max_optin) return cudaErrorInvalidValue;
-        e = cudaFuncSetAttribute(umma_pair_kernel<MODE, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_optin);
-        if (e != cudaSuccess) return e;
-        configured[dev] = max_optin;
-    }
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (smem > static_cast<size_t>(max_optin[dev])) return cudaErrorInvalidValue;
     umma_pair_kernel<MODE, F8><<<grid, NUM_THREADS, smem, st>>>(mr, mw, mt, args);
     return cudaGetLastError();
 }
@@ -593,8 +645,11 @@ PairArgs swiglu_args(int64_t rows_cap, const int32_t* offsets, int N, int d, int
     a.n_groups = N;
     a.kdim = d;
     a.n_out = I;
-    a.ntiles = (I + HALF_M - 1) / HALF_M;  // 128 features (gate + up) per row tile
+    // 128 features (gate + up) per accumulator; when I allows, a row tile covers 256 features
+    // in both accumulators (wide), which halves the row-operand reads per FLOP
     a.tile_cols = HALF_M;
+    a.wide = (I % (2 * HALF_M) == 0) ? 1 : 0;
+    a.ntiles = a.wide ? I / (2 * HALF_M) : (I + HALF_M - 1) / HALF_M;
     a.b_group_rows = 2 * I;
     a.up_off = I;
     a.s_tiles = (I + 2 * HALF_M - 1) / (2 * HALF_M);  // 256 features per weight tile
@@ -649,8 +704,12 @@ PairArgs down_args(int64_t rows_cap, const int32_t* offsets, int N, int d, int I
     a.n_groups = N;
     a.kdim = I;
     a.n_out = d;
-    a.ntiles = (d + 2 * HALF_M - 1) / (2 * HALF_M);  // 256 output features per row tile
+    // 256 output features per accumulator. Wide row tiles (512 features) measured slower here:
+    // with K = I the main loop of a tile is short, and the unoverlapped epilogue of a wide tile
+    // costs more than the row-operand bytes it saves
     a.tile_cols = 2 * HALF_M;
+    a.wide = 0;
+    a.ntiles = (d + 2 * HALF_M - 1) / (2 * HALF_M);
     a.b_group_rows = d;
     a.up_off = 0;
     a.s_tiles = (d + 2 * HALF_M - 1) / (2 * HALF_M);

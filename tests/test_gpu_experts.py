@@ -52,11 +52,16 @@ def test_grouped_gemms_all_rows(cuda_device, name):
 
 def test_grouped_gemms_ragged_group_sizes(cuda_device):
     """Group sizes around the 128-row tile (0, 1, 127, 128, 129, 255, 256, 257, ...), gate/up
-    width I = 128 and I = 64 (a half tile), d = 256 and 192 (down tile of 64)."""
+    width I = 128 and I = 64 (a half tile), d = 256 and 192 (down tile of 64); and gate/up widths
+    whose row tiles span both accumulators (I a multiple of 256: I = 512 and 768, with d = 1024
+    and 1536), with group sizes on both sides of every tile rule (cold below 128 / 256 rows, a
+    padded 128..255-row remainder, leftover rows below 128 after full 256-row tiles)."""
     rng = np.random.default_rng(4)
     for (d, I, sizes) in [(256, 128, [0, 1, 127, 128, 129, 0, 255, 256, 257, 3]),
                           (192, 64, [5, 0, 0, 300, 1, 64]),
-                          (128, 192, [130, 2, 0, 77])]:
+                          (128, 192, [130, 2, 0, 77]),
+                          (1024, 512, [0, 1, 64, 127, 128, 129, 255, 256, 257, 383, 384, 511, 512, 640, 1000]),
+                          (1536, 768, [300, 3, 0, 513, 128, 70])]:
         N = len(sizes)
         M = int(np.sum(sizes))
         T, K = M, 1
