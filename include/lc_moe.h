@@ -214,6 +214,38 @@ int lc_moe_expert_ffn(const lc_moe_shape* s, const void* x_perm, const int32_t* 
 int lc_moe_combine(const lc_moe_shape* s, const void* x, const void* y, const float* gate,
                    const int32_t* pair_row, void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- expert parallelism ---------------------------------------------------------------------
+ * The pages deploy the layer with its experts spread over GPUs (LongCat-Flash llm-wiki entity
+ * page, section 2.2 ScMoE: expert-parallel dispatch and combine; section 5: multi-GPU
+ * deployments). With G ranks, rank r holds FFN experts [r N/G, (r+1) N/G). Each rank routes and
+ * groups its own tokens (lc_moe_route / lc_moe_permute over all N experts), sends every rank the
+ * contiguous slice of its grouped rows that belongs to that rank's experts (an all-to-all; picks
+ * of zero-computation experts, E_i(x) = x, stay on their rank), runs the grouped GEMMs of its own
+ * experts on the rows it received, returns each output row to its source (the inverse
+ * all-to-all) and combines as lc_moe_combine does. The two calls below are the local step
+ * between the exchanges; the exchanges themselves are the caller's (NCCL through
+ * torch.distributed in the Python binding). */
+
+/* Expert-major order of rows received source-major.
+ *   cnt     [G, n_local] int32 (device): rows source rank s sent for local expert e; the rows
+ *           arrived ordered by source, then expert, then the source's token order
+ *   perm    [m_cap] int32 (device): perm[i] = arrival index of the i-th row in expert-major
+ *           order (expert, then source rank, then arrival order); M = sum(cnt) entries written
+ *   offsets [n_local + 1] int32 (device): local expert e owns rows [offsets[e], offsets[e+1])
+ *   ws      status only (LC_MOE_OP_STATUS bytes); M > m_cap or a negative count sets
+ *           LC_MOE_DEV_IDX_RANGE (entries past m_cap are not written).
+ * Needs G * n_local <= 2048 (else LC_MOE_ERR_UNSUPPORTED_SHAPE). */
+int lc_moe_ep_regroup_plan(const int32_t* cnt, int32_t G, int32_t n_local, int32_t* perm, int64_t m_cap,
+                           int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
+
+/* Row copy through an index map, rows of row_bytes bytes (a multiple of 16; 16-byte aligned):
+ *   scatter = 0: dst[i] = src[map[i]]   (gather: received rows into expert-major order)
+ *   scatter = 1: dst[map[i]] = src[i]   (scatter: expert outputs back into arrival order)
+ * for i < n; map must be a permutation of [0, n) (an entry outside it sets LC_MOE_DEV_IDX_RANGE
+ * in the status word of ws and that row is skipped). ws: status only. */
+int lc_moe_copy_rows(const void* src, void* dst, const int32_t* map, int64_t n, int32_t row_bytes,
+                     int32_t scatter, void* ws, size_t ws_bytes, void* stream);
+
 /* lc_moe_permute_noalloc -- lc_moe_permute for callers that cannot allocate device memory: for
  * example code running inside an engine whose memory planner hands out all device memory up
  * front and refuses later requests, or a caller with no workspace of its own to pass. The paper

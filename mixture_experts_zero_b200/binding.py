@@ -31,7 +31,7 @@ EXPORTED = (
     "lc_moe_read_status", "lc_moe_router_logits", "lc_moe_topk", "lc_moe_expert_hist",
     "lc_moe_permute", "lc_moe_expert_ffn", "lc_moe_combine", "lc_moe_permute_noalloc",
     "lc_moe_quantize_e4m3", "lc_moe_forward_fp8", "lc_moe_forward_fp8_timed",
-    "lc_moe_check_wait_timeout",
+    "lc_moe_check_wait_timeout", "lc_moe_ep_regroup_plan", "lc_moe_copy_rows",
 )
 
 
@@ -91,6 +91,8 @@ def _configure(L: ctypes.CDLL) -> ctypes.CDLL:
     L.lc_moe_forward_fp8.argtypes = fwd8
     L.lc_moe_forward_fp8_timed.argtypes = fwd8 + [ctypes.POINTER(P)]
     L.lc_moe_check_wait_timeout.argtypes = [P, SZ, P]
+    L.lc_moe_ep_regroup_plan.argtypes = [P, I32, I32, P, I64, P, P, SZ, P]
+    L.lc_moe_copy_rows.argtypes = [P, P, P, I64, I32, I32, P, SZ, P]
     return L
 
 
@@ -450,3 +452,47 @@ def lc_moe_permute_noalloc(idx, N: int, E: int, x=None, d: int = 64, want_rows: 
                                          _ptr(row_token), _ptr(pair_row), _ptr(x_perm), _ptr(status),
                                          _stream(stream)), "lc_moe_permute_noalloc")
     return offsets, row_token, pair_row, x_perm
+
+
+# ------------------------------------------------------------------- expert parallelism --
+
+def _status_ws(device):
+    return new_workspace(Shape(1, 64, 1, 0, 1, 64), OP_STATUS, device)
+
+
+def lc_moe_ep_regroup_plan(cnt, m_cap: int | None = None, perm=None, offsets=None, ws=None, stream=None):
+    """Expert-major order of rows received source-major. ``cnt`` int32 [G, n_local] (device):
+    rows source s sent for local expert e. Returns (perm [M] int32, offsets [n_local + 1] int32)
+    with M = cnt.sum() (m_cap, when given, is the length of ``perm``)."""
+    if cnt.dtype != torch.int32 or cnt.dim() != 2 or not cnt.is_cuda or not cnt.is_contiguous():
+        raise ValueError("cnt: expected a contiguous int32 CUDA tensor [G, n_local]")
+    G, n_local = cnt.shape
+    if m_cap is None:
+        m_cap = int(cnt.sum().item())
+    if perm is None:
+        perm = torch.empty(max(m_cap, 1), dtype=torch.int32, device=cnt.device)
+    if offsets is None:
+        offsets = torch.empty(n_local + 1, dtype=torch.int32, device=cnt.device)
+    _need(offsets, torch.int32, (n_local + 1,), "offsets")
+    if ws is None:
+        ws = _status_ws(cnt.device)
+    _check(_lib().lc_moe_ep_regroup_plan(_ptr(cnt), G, n_local, _ptr(perm), int(m_cap), _ptr(offsets),
+                                         _ptr(ws), ws.numel(), _stream(stream)), "lc_moe_ep_regroup_plan")
+    return perm[:m_cap], offsets
+
+
+def lc_moe_copy_rows(src, index, scatter: bool = False, out=None, ws=None, stream=None):
+    """Rows of ``src`` [n, ...] moved through the permutation ``index`` [n] int32:
+    out[i] = src[index[i]] (gather) or out[index[i]] = src[i] (scatter)."""
+    n = index.shape[0]
+    if src.shape[0] < n or not src.is_cuda or not src.is_contiguous():
+        raise ValueError("src: expected a contiguous CUDA tensor with at least len(index) rows")
+    _need(index, torch.int32, (n,), "index")
+    row_bytes = src[0].numel() * src.element_size() if src.shape[0] else 16
+    if out is None:
+        out = torch.empty((n,) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    if ws is None:
+        ws = _status_ws(src.device)
+    _check(_lib().lc_moe_copy_rows(_ptr(src), _ptr(out), _ptr(index), n, row_bytes, 1 if scatter else 0,
+                                   _ptr(ws), ws.numel(), _stream(stream)), "lc_moe_copy_rows")
+    return out

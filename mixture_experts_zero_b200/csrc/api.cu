@@ -183,23 +183,25 @@ int forward_impl(const lc_moe_shape* s, const void* x, const void* wr, const flo
 }  // namespace
 
 const DevInfo* current_device_info() {
-    static DevInfo infos[64];
-    static std::once_flag flags[64];
-    static bool valid[64];
+    static PerDeviceOnce query;
+    static DevInfo infos[PerDeviceOnce::kMaxDevices];
+    const cudaError_t e = query.run([](int dev) {
+        int major = 0, minor = 0, sms = 0;
+        cudaError_t r = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (r == cudaSuccess) r = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (r == cudaSuccess) r = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (r == cudaSuccess) {
+            infos[dev].sm_count = sms;
+            infos[dev].ok_sm100 = (major == 10 && minor == 0);
+        }
+        return r;
+    });
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    if (e != cudaSuccess || cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
         return nullptr;
     }
-    std::call_once(flags[dev], [dev] {
-        int major = 0, minor = 0, sms = 0;
-        valid[dev] = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
-                     cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
-                     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess;
-        infos[dev].sm_count = sms;
-        infos[dev].ok_sm100 = (major == 10 && minor == 0);
-    });
-    return valid[dev] ? &infos[dev] : nullptr;
+    return &infos[dev];
 }
 
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
@@ -438,6 +440,34 @@ int lc_moe_combine(const lc_moe_shape* s, const void* x, const void* y, const fl
     if (s->T == 0) return LC_MOE_OK;
     LC_TRY(device_ok());
     LC_CUDA(launch_combine(x, y, gate, pair_row, s->T, s->d, s->K, out, static_cast<cudaStream_t>(stream)));
+    return LC_MOE_OK;
+}
+
+int lc_moe_ep_regroup_plan(const int32_t* cnt, int32_t G, int32_t n_local, int32_t* perm, int64_t m_cap,
+                           int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
+    if (!cnt || !offsets || !ws || (m_cap > 0 && !perm)) return LC_MOE_ERR_INVALID_ARG;
+    if (G < 1 || n_local < 1 || m_cap < 0) return LC_MOE_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(G) * n_local > 2048 || m_cap >= (int64_t(1) << 31)) return LC_MOE_ERR_UNSUPPORTED_SHAPE;
+    if (ws_bytes < kStatusBytes) return LC_MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(ws)) return LC_MOE_ERR_MISALIGNED;
+    LC_TRY(device_ok());
+    LC_CUDA(launch_regroup_plan(cnt, G, n_local, perm, m_cap, offsets, at<uint32_t>(ws, 0),
+                                static_cast<cudaStream_t>(stream)));
+    return LC_MOE_OK;
+}
+
+int lc_moe_copy_rows(const void* src, void* dst, const int32_t* map, int64_t n, int32_t row_bytes,
+                     int32_t scatter, void* ws, size_t ws_bytes, void* stream) {
+    if (n < 0 || row_bytes <= 0 || row_bytes % 16 || (scatter != 0 && scatter != 1) || !ws)
+        return LC_MOE_ERR_INVALID_ARG;
+    if (n > 0 && (!src || !dst || !map)) return LC_MOE_ERR_INVALID_ARG;
+    if (ws_bytes < kStatusBytes) return LC_MOE_ERR_WORKSPACE_TOO_SMALL;
+    for (const void* p : {src, static_cast<const void*>(dst), static_cast<const void*>(ws)})
+        if (p && !aligned16(p)) return LC_MOE_ERR_MISALIGNED;
+    if (n == 0) return LC_MOE_OK;
+    LC_TRY(device_ok());
+    LC_CUDA(launch_copy_rows(src, dst, map, n, row_bytes, scatter, at<uint32_t>(ws, 0),
+                             static_cast<cudaStream_t>(stream)));
     return LC_MOE_OK;
 }
 
