@@ -58,10 +58,7 @@ namespace {
 
 constexpr int HALF_M = 128;                 // A rows per CTA
 constexpr int BK = 64;                      // 64 bf16 = 128 bytes = one swizzle row
-constexpr int STAGES = 4;
-constexpr int A_BYTES = HALF_M * BK * 2;    // 16 KB
-constexpr int B_SLOT = 2 * A_BYTES;         // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_SLOT;
+constexpr int A_BYTES = HALF_M * BK * 2;    // 16 KB: one 128-row operand box of a k-step
 constexpr int TMEM_COLS = 512;
 constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;              // warps 4..11: two epilogue groups of four warps
@@ -69,6 +66,17 @@ constexpr int TOK_BOX = 32;                 // token rows per TMA box of a weigh
 constexpr int TOK_ROUND = 2 * TOK_BOX;      // weight-tile N is a multiple of this
 
 enum Mode : int { MODE_SWIGLU = 1, MODE_DOWN = 2 };
+
+// Shared-memory ring of each GEMM. GEMM 1 stages hold the row box and two weight boxes (a wide
+// row tile's two accumulators, or a weight tile's gate and up rows plus up to 64 token rows): 48 KB
+// in 4 stages. GEMM 2 stages hold two boxes (rows and weights, or weights and up to 128 token rows):
+// 32 KB, so the same shared memory holds 6 stages, half again the bytes in flight of the weight
+// stream that the cold experts' tiles are.
+template <int MODE>
+struct Ring {
+    static constexpr int stages = MODE == MODE_DOWN ? 6 : 4;
+    static constexpr int bytes = MODE == MODE_DOWN ? 2 * A_BYTES : 3 * A_BYTES;
+};
 
 struct PairArgs {
     const int32_t* offsets;  // [n_groups + 1] row offsets
@@ -99,8 +107,10 @@ struct PairArgs {
 constexpr int XPOSE_ROW = 64;
 constexpr int XPOSE_WARP = 32 * XPOSE_ROW;
 
+template <int MODE>
 struct Layout {
-    static constexpr int bars_off = STAGES * STAGE_BYTES;
+    static constexpr int STAGES = Ring<MODE>::stages;
+    static constexpr int bars_off = STAGES * Ring<MODE>::bytes;
     static constexpr int n_bars = 2 * STAGES + 5;  // full, empty, tfull[2], tempty[2], drain
     static constexpr int misc_off = bars_off + n_bars * 8;
     static constexpr int xpose_off = (misc_off + 16 + 127) & ~127;
@@ -166,6 +176,9 @@ template <int MODE, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     umma_pair_kernel(const __grid_constant__ CUtensorMap mapRows, const __grid_constant__ CUtensorMap mapW,
                      const __grid_constant__ CUtensorMap mapTok, const PairArgs g) {
+    constexpr int STAGES = Ring<MODE>::stages;
+    constexpr int STAGE_BYTES = Ring<MODE>::bytes;
+    using Layout = ::lcmoe::Layout<MODE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -607,7 +620,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 template <int MODE, bool F8>
 cudaError_t launch_pair(const CUtensorMap& mr, const CUtensorMap& mw, const CUtensorMap& mt,
                         const PairArgs& args, int grid, cudaStream_t st) {
-    const size_t smem = Layout::bytes(args.n_groups);
+    // a GEMM 2 stage holds two boxes: its row tiles are never wide
+    if (MODE == MODE_DOWN && args.wide) return cudaErrorInvalidValue;
+    const size_t smem = Layout<MODE>::bytes(args.n_groups);
     // once per device: allow the kernel the device's whole opt-in shared memory
     static PerDeviceOnce setup;
     static int max_optin[PerDeviceOnce::kMaxDevices];
