@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(TOPK_THREADS)
     float* s_bias = reinterpret_cast<float*>(smem_i + E);      // [E]
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    float* s_score = s_bias + E + warp * E;                     // [8][E]: this warp's token scores
     const bool do_hist = counts != nullptr;
     for (int i = threadIdx.x; i < E; i += TOPK_THREADS) {
         s_hist[i] = 0;
@@ -124,6 +125,7 @@ __global__ void __launch_bounds__(TOPK_THREADS)
             ku[j] = 0;
             if (i < E) {
                 v[j] = __fdiv_rn(v[j], S);
+                s_score[i] = v[j];
                 const float key = __fadd_rn(v[j], s_bias[i]);
                 nan_key |= (key != key);
                 const uint32_t kb = __float_as_uint(key);
@@ -139,46 +141,50 @@ __global__ void __launch_bounds__(TOPK_THREADS)
             }
             continue;
         }
-        // K rounds of warp arg-max over (key, index); each lane keeps its best two untaken
-        // (key, index, score) and rescans only when both are taken.
+        // K rounds of warp arg-max over (key, index); each lane keeps its best three untaken keys
+        // (with their indices) and rescans only when all three are taken. The scores are kept in
+        // this warp's shared-memory row, read back for the K winners only.
         uint64_t taken = 0;
-        uint32_t k1 = 0, k2 = 0;
-        int i1 = 0x7fffffff, i2 = 0x7fffffff;
-        float s1 = 0.0f, s2 = 0.0f;
-        auto top2 = [&]() {
-            k1 = k2 = 0;
-            i1 = i2 = 0x7fffffff;
+        uint32_t k1 = 0, k2 = 0, k3 = 0;
+        int i1 = 0x7fffffff, i2 = 0x7fffffff, i3 = 0x7fffffff;
+        auto top3 = [&]() {
+            k1 = k2 = k3 = 0;
+            i1 = i2 = i3 = 0x7fffffff;
 #pragma unroll
             for (int j = 0; j < VPL; ++j) {
                 const int i = lane + 32 * j;
-                if (!((taken >> j) & 1ull)) {  // ku = 0 (past E) never wins
-                    if (ku[j] > k1) {
-                        k2 = k1; i2 = i1; s2 = s1;
-                        k1 = ku[j]; i1 = i; s1 = v[j];
-                    } else if (ku[j] > k2) {
-                        k2 = ku[j]; i2 = i; s2 = v[j];
+                const uint32_t kj = ((taken >> j) & 1ull) ? 0u : ku[j];  // ku = 0 (past E) never wins
+                if (kj > k3) {
+                    if (kj > k2) {
+                        k3 = k2; i3 = i2;
+                        if (kj > k1) {
+                            k2 = k1; i2 = i1;
+                            k1 = kj; i1 = i;
+                        } else {
+                            k2 = kj; i2 = i;
+                        }
+                    } else {
+                        k3 = kj; i3 = i;
                     }
                 }
             }
         };
-        top2();
+        top3();
         int my_idx = 0;
-        float my_s = 0.0f;
         for (int r = 0; r < K; ++r) {
             const uint32_t m = __reduce_max_sync(0xffffffffu, k1);
             const int w = __reduce_min_sync(0xffffffffu, k1 == m ? static_cast<uint32_t>(i1) : 0x7fffffffu);
-            const float ws = __shfl_sync(0xffffffffu, s1, w & 31);
-            if (lane == r) {
-                my_idx = w;
-                my_s = ws;
-            }
+            if (lane == r) my_idx = w;
             if ((w & 31) == lane) {
                 taken |= 1ull << (w >> 5);
-                k1 = k2; i1 = i2; s1 = s2;
-                k2 = 0; i2 = 0x7fffffff;
-                if (k1 == 0) top2();
+                k1 = k2; i1 = i2;
+                k2 = k3; i2 = i3;
+                k3 = 0; i3 = 0x7fffffff;
+                if (k1 == 0) top3();
             }
         }
+        __syncwarp();
+        const float my_s = lane < K ? s_score[my_idx] : 0.0f;
         // renormalise over the K chosen, summing in rank order
         float Q = 0.0f;
         for (int r = 0; r < K; ++r) Q = __fadd_rn(Q, __shfl_sync(0xffffffffu, my_s, r));
@@ -206,7 +212,14 @@ cudaError_t launch_topk_t(const float* logits, const float* bias, int T, int E, 
     const int cap = sm_count * 4;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    const size_t smem = 2 * static_cast<size_t>(E) * sizeof(int32_t);
+    // histogram, biases and one score row per warp: 80 KB at E = 2048
+    const size_t smem = (2 + warps) * static_cast<size_t>(E) * sizeof(int32_t);
+    static PerDeviceOnce setup;
+    const cudaError_t e = setup.run([](int) {
+        return cudaFuncSetAttribute(topk_kernel<VPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>((2 + TOPK_THREADS / 32) * 32 * VPL * sizeof(int32_t)));
+    });
+    if (e != cudaSuccess) return e;
     topk_kernel<VPL><<<blocks, TOPK_THREADS, smem, st>>>(logits, bias, T, E, K, idx, gate, counts,
                                                           status);
     return cudaGetLastError();
