@@ -332,6 +332,8 @@ def run_ours(args):
     }
     med = np.median(stage_ms, axis=0)
     mean = np.mean(stage_ms, axis=0)
+    # the grouping is one kernel for a batch of at most 256 tokens, three above
+    n_kernels = sum(KERNELS_PER_STAGE) - (2 if T <= 256 else 0)
     stages = {}
     for j, name in enumerate(STAGES):
         bound, work = alg[name]
@@ -386,9 +388,9 @@ def run_ours(args):
                 "d2h_bytes_per_step": int(out.numel() * 2), "steps": e2e_steps_n,
                 "copies": "pinned host x -> device and out -> pinned host every step, on a copy "
                           "stream overlapping the neighbouring steps' compute"},
-        "gpu_launches": int(args.steps * (sum(KERNELS_PER_STAGE) + 1 + (2 if f8 else 0))),
+        "gpu_launches": int(args.steps * (n_kernels + 1 + (2 if f8 else 0))),
         "gpu_launches_note": "kernels of this library inside the device-timed region: "
-                             f"{sum(KERNELS_PER_STAGE) + (2 if f8 else 0)} per forward "
+                             f"{n_kernels + (2 if f8 else 0)} per forward "
                              f"{'(incl. the token-row and H-row quantisers) ' if f8 else ''}+ 1 bias update, per step",
         "clocks": ClockSampler.summarize(clock_rows),
     }
@@ -725,7 +727,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill",
-                    choices=["prefill", "decode", "small", "tiny", "prefill_ncu", "route_ncu"])
+                    choices=["prefill", "decode", "small", "tiny", "prefill_ncu", "route_ncu", "decode_ncu"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-route-tokens", type=int, default=None,
                     help="tokens the CPU baseline routes (default: the whole batch)")

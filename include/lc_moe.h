@@ -120,6 +120,13 @@ void lc_moe_set_wait_limit_ns(uint64_t limit_ns);
  * lc_moe_read_status then returns LC_MOE_ERR_TIMEOUT. ws: status only (LC_MOE_OP_STATUS bytes). */
 int lc_moe_check_wait_timeout(void* ws, size_t ws_bytes, void* stream);
 
+/* Test switch of the abort path of the grouped expert GEMMs (no entry point of its own): with the
+ * environment variable LC_MOE_DEBUG_GEMM_ABORT_KSTEP=k set when a GEMM is launched, its MMA
+ * issuers give up before their k-th k-step as if a pipeline wait had run out. The other roles of
+ * each CTA pair then leave through the abort flag or their own bounded waits (about one wait limit
+ * of device time), wait for the copies and MMAs they issued, and free TMEM; the status word gets
+ * LC_MOE_DEV_WAIT_TIMEOUT and the GEMM outputs are incomplete. Unset in normal use. */
+
 /*
  * lc_moe_forward -- the whole MoE layer (MoE equation, section 2.1).
  *   x      [T, d]   bf16   token activations x_t

@@ -13,6 +13,7 @@
 //   scatter : the row of pick (t, r) of expert e is
 //             offsets[e] + base[b][e] + popc(mask of e restricted to tokens before t in block b),
 //             so rows of an expert are in ascending token order. Writes pair_row and row_token.
+//   single  : a batch of at most 256 tokens (one block) does all three in one launch.
 //   gather  : per token, x_t is read once into shared memory with one bulk async copy and
 //             written to each of its FFN rows with one bulk store per row (rows above 25 KB:
 //             one warp per token copies 16-byte vectors through registers); x_t is read once
@@ -148,6 +149,78 @@ __global__ void __launch_bounds__(PB)
             int rank = __popc(mask[e * MASK_WORDS + w] & below);
             for (int j = 0; j < w; ++j) rank += __popc(mask[e * MASK_WORDS + j]);
             row = offsets[e] + base[static_cast<int64_t>(blockIdx.x) * N + e] + rank;
+            row_token[row] = t;
+        }
+        pair_row[static_cast<int64_t>(t) * K + r] = row;
+    }
+}
+
+// All of it in one block when the batch is one block of tokens (T <= 256, decode-sized batches):
+// masks and counts as in perm_count_kernel, the exclusive scan of the counts over the experts in
+// shared memory, and the scatter of perm_scatter_kernel with every base 0; one launch instead of
+// three.
+__global__ void __launch_bounds__(PB)
+    perm_single_kernel(const int32_t* __restrict__ idx, int T, int K, int N, int E,
+                       int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
+                       int32_t* __restrict__ pair_row, uint32_t* __restrict__ status) {
+    extern __shared__ uint32_t mask[];              // [N][MASK_WORDS]
+    int32_t* offs = reinterpret_cast<int32_t*>(mask + N * MASK_WORDS);  // [N]
+    __shared__ int32_t warp_sums[PB / 32];
+    __shared__ int32_t carry;
+    for (int i = threadIdx.x; i < N * MASK_WORDS; i += PB) mask[i] = 0;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    const bool bad = build_masks(idx, T, K, N, E, mask, status);
+    if (__syncthreads_or(bad) && threadIdx.x == 0) set_status(status, LC_MOE_DEV_IDX_RANGE);
+    // exclusive scan of the per-expert counts, PB experts at a time
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int e0 = 0; e0 < N; e0 += PB) {
+        const int e = e0 + threadIdx.x;
+        int v = 0;
+        if (e < N) {
+#pragma unroll
+            for (int w = 0; w < MASK_WORDS; ++w) v += __popc(mask[e * MASK_WORDS + w]);
+        }
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+        }
+        if (lane == 31) warp_sums[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int ws = lane < PB / 32 ? warp_sums[lane] : 0;
+            int wi = ws;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, wi, o);
+                if (lane >= o) wi += u;
+            }
+            if (lane < PB / 32) warp_sums[lane] = wi - ws;  // exclusive prefix of warp totals
+        }
+        __syncthreads();
+        const int excl = carry + warp_sums[warp] + incl - v;
+        if (e < N) {
+            offs[e] = excl;
+            offsets[e] = excl;
+        }
+        __syncthreads();
+        if (threadIdx.x == PB - 1) carry = excl + v;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) offsets[N] = carry;
+    const int t = threadIdx.x;
+    if (t >= T) return;
+    const int w = threadIdx.x >> 5;
+    const uint32_t below = (1u << (threadIdx.x & 31)) - 1u;
+    for (int r = 0; r < K; ++r) {
+        const int e = idx[static_cast<int64_t>(t) * K + r];
+        int row = -1;
+        if (e >= 0 && e < N) {
+            int rank = __popc(mask[e * MASK_WORDS + w] & below);
+            for (int j = 0; j < w; ++j) rank += __popc(mask[e * MASK_WORDS + j]);
+            row = offs[e] + rank;
             row_token[row] = t;
         }
         pair_row[static_cast<int64_t>(t) * K + r] = row;
@@ -322,14 +395,22 @@ cudaError_t launch_permute(const int32_t* idx, int T, int K, int N, int E, int32
     const size_t mask_bytes = static_cast<size_t>(N) * MASK_WORDS * sizeof(uint32_t);
     static PerDeviceOnce setup;
     cudaError_t e = setup.run([](int) {
-        // masks of up to 2048 experts take 64 KB of shared memory
+        // masks of up to 2048 experts take 64 KB of shared memory (plus their offsets: 72 KB)
         cudaError_t r = cudaFuncSetAttribute(perm_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              2048 * MASK_WORDS * 4);
+        if (r != cudaSuccess) return r;
+        r = cudaFuncSetAttribute(perm_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 2048 * (MASK_WORDS + 1) * 4);
         if (r != cudaSuccess) return r;
         return cudaFuncSetAttribute(perm_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     2048 * MASK_WORDS * 4);
     });
     if (e != cudaSuccess) return e;
+    if (nblk <= 1) {
+        perm_single_kernel<<<1, PB, static_cast<size_t>(N) * (MASK_WORDS + 1) * sizeof(uint32_t), st>>>(
+            idx, T, K, N, E, offsets, row_token, pair_row, status);
+        return cudaGetLastError();
+    }
     if (nblk > 0) {
         perm_count_kernel<<<nblk, PB, mask_bytes, st>>>(idx, T, K, N, E, cnt, status);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -48,6 +48,7 @@
 // records LC_MOE_DEV_WAIT_TIMEOUT, drains in-flight copies and MMAs, and frees TMEM.
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -99,6 +100,7 @@ struct PairArgs {
     int wide;                // row tiles span two accumulators (2 * tile_cols output columns)
     const float* row_scale;  // E4M3 GEMM 1: scale of each grouped row [rows_cap]
     const float* w_scale;    // E4M3 GEMM 1: scale of each weight row [n_groups * b_group_rows]
+    int64_t abort_kstep;     // test switch: the MMA issuer gives up before this k-step (< 0: never)
 };
 
 // Epilogue transpose tile of one warp: 32 rows x 32 features (bf16), 64 bytes per row, its four
@@ -150,7 +152,10 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint6
     return true;
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+// silu(g) * u. The quotient is the fast division (within 2 ulp of fp32, and 0 once 1 + e^-g
+// passes 2^126, where silu(g) is below 2^-119): the IEEE division routine made the SwiGLU
+// epilogue three times longer (15 against 5 us per 128 x 128 block), and H is rounded to bf16.
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 template <bool F8>
 __device__ __forceinline__ void mma_step(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
@@ -390,6 +395,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         uint32_t ph = 0;
         AccSchedule sched;
         bool ok = true;
+        int64_t ksteps = 0;
         for (int tile = cluster; tile < total && ok; tile += n_clusters) {
             const Tile tl = decode(tile);
             const uint32_t idesc = F8 ? idesc_e4m3_f32(2 * HALF_M, tl.swap ? tl.ntok : 2 * HALF_M)
@@ -402,6 +408,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const int acc = tl.wide ? 0 : sched.next;
             const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
             for (int kb = 0; kb < nk; ++kb) {
+                if (ksteps++ == g.abort_kstep) {
+                    // as if this stage's wait had run out: the abort and drain paths of every role
+                    *abort_flag = 1;
+                    set_status(g.status, LC_MOE_DEV_WAIT_TIMEOUT);
+                    ok = false;
+                    break;
+                }
                 if (!mbar_wait(&full[s], ph, g.wait_ns, abort_flag, g.status)) {
                     ok = false;
                     break;
@@ -471,11 +484,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 const int64_t grow = tl.row0 + r;
                 const bool valid = r < tl.rows && grow < g.rows_cap;
                 if (MODE == MODE_SWIGLU) {
-                    for (int c = 0; c < HALF_M; c += 32) {
-                        uint32_t gv[32], uv[32];
-                        tmem_ld_32x32b_x32(tb + c, gv);
-                        tmem_ld_32x32b_x32(tb + HALF_M + c, uv);
+                    // the next 32 columns' TMEM loads are in flight while this block is computed
+                    uint32_t gbuf[2][32], ubuf[2][32];
+                    tmem_ld_32x32b_x32(tb, gbuf[0]);
+                    tmem_ld_32x32b_x32(tb + HALF_M, ubuf[0]);
+#pragma unroll
+                    for (int ci = 0; ci < HALF_M / 32; ++ci) {
+                        const int c = ci * 32;
                         tmem_ld_wait();
+                        if (ci + 1 < HALF_M / 32) {
+                            tmem_ld_32x32b_x32(tb + c + 32, gbuf[(ci + 1) & 1]);
+                            tmem_ld_32x32b_x32(tb + HALF_M + c + 32, ubuf[(ci + 1) & 1]);
+                        }
+                        uint32_t (&gv)[32] = gbuf[ci & 1];
+                        uint32_t (&uv)[32] = ubuf[ci & 1];
                         const int f0 = fbase + c;
                         if (valid && f0 < g.n_out) {
                             if (F8) {
@@ -644,6 +666,18 @@ cudaError_t launch_pair(const CUtensorMap& mr, const CUtensorMap& mw, const CUte
 
 int pair_grid(const DevInfo* di) { return (di->sm_count / 2) * 2; }
 
+// The k-step before which the MMA issuer of every grouped-GEMM launch gives up as if a wait had
+// run out, from the environment variable LC_MOE_DEBUG_GEMM_ABORT_KSTEP (unset in normal use: never).
+// It exists for the device test of the abort path: the other roles then leave through the abort
+// flag or their own bounded waits, drain what they issued and free TMEM.
+int64_t debug_abort_kstep() {
+    const char* v = std::getenv("LC_MOE_DEBUG_GEMM_ABORT_KSTEP");
+    if (!v || !*v) return -1;
+    char* end = nullptr;
+    const long long k = std::strtoll(v, &end, 10);
+    return (end && *end == '\0' && k >= 0) ? static_cast<int64_t>(k) : -1;
+}
+
 }  // namespace
 
 namespace {
@@ -655,6 +689,7 @@ PairArgs swiglu_args(int64_t rows_cap, const int32_t* offsets, int N, int d, int
     a.out = static_cast<__nv_bfloat16*>(h);
     a.status = status;
     a.wait_ns = wait_limit_ns();
+    a.abort_kstep = debug_abort_kstep();
     a.rows_cap = rows_cap;
     a.ldo = I;
     a.n_groups = N;
@@ -714,6 +749,7 @@ PairArgs down_args(int64_t rows_cap, const int32_t* offsets, int N, int d, int I
     a.out = static_cast<__nv_bfloat16*>(y);
     a.status = status;
     a.wait_ns = wait_limit_ns();
+    a.abort_kstep = debug_abort_kstep();
     a.rows_cap = rows_cap;
     a.ldo = d;
     a.n_groups = N;

@@ -61,6 +61,9 @@ WORKLOADS = {
     # captures of the router GEMM, the top-K and the grouping at full routing width
     "route_ncu": Workload("route_ncu", T=8192, d=6144, N=512, Z=256, K=12, K_e=8, I=64, seed=3,
                           router="zipf"),
+    # LongCat-Flash router shape at decode batch size (T = 128) with 64-wide experts (~0.8 GB on
+    # the device): profiler captures of the small-batch routing and one-launch grouping
+    "decode_ncu": Workload("decode_ncu", T=128, d=6144, N=512, Z=256, K=12, K_e=8, I=64, seed=2),
     # bias-control loop: 200 fresh batches of 8192 tokens, routing only
     "bias_loop": Workload("bias_loop", T=8192, d=6144, N=512, Z=256, K=12, K_e=8, I=2048,
                           seed=4, steps=200),
