@@ -591,12 +591,17 @@ def run_sweep(args):
         I=2048) with c rows for each of n experts, against max(6*M*d*I FLOP / sustained TC peak,
         (3*n*d*I + 2*M*(2d+I)) * 2 bytes / HBM).
     hist: the expert-count histogram over idx[2^24, 12] (805 MB of int32), against HBM.
-    control: the bias-control loop at LongCat-Flash shape (run_control)."""
+    control: the bias-control loop at LongCat-Flash shape (run_control).
+    ffn_subset: the expert GEMMs on every 8th FFN expert of the prefill workload's routing
+        (run_ffn_subset)."""
     import torch
     from mixture_experts_zero_b200 import binding as B
 
     if args.sweep == "control":
         run_control(args)
+        return
+    if args.sweep == "ffn_subset":
+        run_ffn_subset(args)
         return
 
     peaks, peak_src = load_peaks()
@@ -654,6 +659,63 @@ def run_sweep(args):
                           "tflops": round(flop / ms / 1e9, 1), "gbs": round(bytes_ / ms / 1e6, 1),
                           "peak_source": peak_src}), flush=True)
         del x, h, y
+
+
+def run_ffn_subset(args, stride: int = 8):
+    """The grouped expert GEMMs (lc_moe_expert_ffn) on a representative eighth of the prefill
+    layer's FFN experts: the prefill batch is routed on the device, the 512 FFN experts are ranked
+    by their row counts, and every 8th of them (ranks 0, 8, 16, ...) keeps its rows, so the 64
+    experts have the full layer's distribution of rows per expert with 1/8 of its weights
+    (4.8 GB) and rows. For profiler captures whose traffic scales to the full layer by the number
+    of experts (x 8). Prints one JSON line: the experts' row counts, M, and the device time of the
+    two GEMMs (median of 8, L2 flushed before each)."""
+    import torch
+    from mixture_experts_zero_b200 import binding as B
+    from mixture_experts_zero_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = inputs.WORKLOADS["prefill"]
+    g = inputs.generator(w.seed, dev)
+    x = inputs.draw_x(w, g, dev)
+    wr = inputs.draw_router(w, g, dev)
+    bias = inputs.draw_bias(w, g, dev)
+    counts = torch.zeros(w.E, dtype=torch.int32, device=dev)
+    idx, _ = B.lc_moe_route(x, wr, bias, w.K, w.N, counts=counts)[:2]
+    c = counts[: w.N].cpu().numpy().astype(np.int64)
+    order = np.argsort(-c, kind="stable")
+    keep = np.sort(order[::stride])
+    sizes = c[keep]
+    n, M = len(keep), int(sizes.sum())
+    # the kept experts' rows: the tokens that picked each of them, grouped by expert
+    idx_h = idx.cpu().numpy()
+    tokens = np.concatenate([np.nonzero((idx_h == e).any(axis=1))[0] for e in keep])
+    xp = x[torch.from_numpy(tokens).to(dev)].contiguous()
+    offsets = torch.from_numpy(np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)).to(dev)
+    gw = torch.Generator(device=dev).manual_seed(w.seed)
+    std = 1.0 / math.sqrt(w.d)
+    w13 = torch.empty(n, 2 * w.I, w.d, dtype=torch.bfloat16, device=dev)
+    w2 = torch.empty(n, w.d, w.I, dtype=torch.bfloat16, device=dev)
+    for e in range(n):
+        w13[e].copy_(torch.randn(2 * w.I, w.d, generator=gw, device=dev) * std)
+        w2[e].copy_(torch.randn(w.d, w.I, generator=gw, device=dev) * std)
+    h = torch.empty(M, w.I, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(M, w.d, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 * 2 ** 20 // 4, device=dev)
+    ts = []
+    for i in range(11):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        B.lc_moe_expert_ffn(xp, offsets, w13, w2, M, 1, h=h, y=y)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ts.append(e0.elapsed_time(e1))
+    ts.sort()
+    print(json.dumps({"sweep": "ffn_subset", "stride": stride, "experts": n, "rows_M": M,
+                      "rows_per_expert": sizes.tolist(), "ms": round(ts[len(ts) // 2], 3),
+                      "weights_gb": round(n * 3 * w.d * w.I * 2 / 1e9, 2)}), flush=True)
 
 
 def run_control(args):
@@ -736,7 +798,7 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=8, help="tokens per reference-arm step")
     ap.add_argument("--experts", choices=["bf16", "fp8"], default="bf16",
                     help="fp8: E4M3 expert projections (lc_moe_forward_fp8)")
-    ap.add_argument("--sweep", choices=["ffn_rows", "hist", "control"], default=None,
+    ap.add_argument("--sweep", choices=["ffn_rows", "hist", "control", "ffn_subset"], default=None,
                     help="run a kernel sweep instead of the step (one GPU)")
     args = ap.parse_args()
     if args.sweep:
