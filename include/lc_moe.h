@@ -264,7 +264,8 @@ int lc_moe_copy_rows(const void* src, void* dst, const int32_t* map, int64_t n, 
  *   - status: optional device uint32 (NULL: not reported) that receives the LC_MOE_DEV_* bits,
  *     OR-ed in; the caller clears it.
  *   - The first call on a device looks up the array's device address; make that first call
- *     before any stream capture.
+ *     before any stream capture (a lookup that fails is returned as LC_MOE_ERR_CUDA and tried
+ *     again by the next call; only a successful one is kept).
  *   - Every call shares the one array: calls that overlap on the GPU (different streams without
  *     ordering, several host threads) race and give wrong groupings. Calls ordered on one stream
  *     are safe; no state is carried from one call to the next.
