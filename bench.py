@@ -451,7 +451,7 @@ def _oracle_combine(w, x_bits, tokens, idx, gate, pairs, Y):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, data, route_tokens: int | None = None, ffn_tokens: int = 256, chunk: int = 64):
+def cpu_baseline(w, data, route_tokens: int | None = None, ffn_tokens: int = 512, chunk: int = 64):
     """The oracle on the host cores, on a bounded sample of the batch, in three timed phases:
     routing (router logits, softmax, biased top-K) of the first ``route_tokens`` tokens (all T by
     default); the SwiGLU experts of every FFN pick of a seeded subset of ``ffn_tokens`` of them,
@@ -488,7 +488,8 @@ def cpu_baseline(w, data, route_tokens: int | None = None, ffn_tokens: int = 256
     threads = oracle.num_threads()
     return {"value": round(value, 3), "unit": UNIT, "cores": threads,
             "cpu": cpu_model(), "host_cpus": os.cpu_count(), "kind": "oracle",
-            "sample": (f"subset-measured: routing of {R} tokens of the {w.name} batch "
+            "sample": (("full batch: " if (R == w.T and F == w.T) else "subset-measured: ")
+                       + f"routing of {R} tokens of the {w.name} batch "
                        f"({t_route:.2f} s), SwiGLU experts of the {len(pairs)} FFN picks of {F} "
                        f"seeded tokens of them ({t_ffn:.2f} s, {len(rows_per_call)} oracle calls "
                        f"of {min(rows_per_call)}-{max(rows_per_call)} rows, every row of up to "
@@ -780,6 +781,33 @@ def run_control(args):
                 "load_max_over_mean_first_last": [round(sp[0], 3), round(sp[-1], 3)],
                 "zero_minus_ffn_mean_bias": zero_bias,
                 "control_step_ms_median": round(ms[len(ms) // 2], 4)}), flush=True)
+    if not args.no_cpu_baseline:
+        print(json.dumps(control_cpu_baseline(w, dev)), flush=True)
+
+
+def control_cpu_baseline(w, dev, steps: int = 2):
+    """The oracle's control step on the host cores: the first ``steps`` steps of the b = 0,
+    mu = 1e-3 loop (same router and tokens as the device run), each timed over router logits in
+    double, softmax + biased top-K + counts, and the bias update."""
+    import oracle
+    from mixture_experts_zero_b200 import inputs
+    g = inputs.generator(w.seed, dev)
+    wr_bits = inputs.bits(inputs.draw_router(w, g, dev))
+    b = np.zeros(w.E, np.float32)
+    secs = []
+    for _ in range(steps):
+        x_bits = inputs.bits(inputs.draw_x(w, g, dev))
+        t0 = time.perf_counter()
+        z = oracle.router_logits(x_bits, wr_bits)
+        _, _, cnt, _ = oracle.route(z, b, w.K)
+        b = oracle.bias_update(b, cnt, w.T, w.N, w.Z, w.K, w.K_e, w.mu)
+        secs.append(time.perf_counter() - t0)
+    step_s = sum(secs) / steps
+    return {"sweep": "control", "impl": "cpu_baseline", "kind": "oracle", "cores": oracle.num_threads(),
+            "cpu": cpu_model(), "host_cpus": os.cpu_count(),
+            "sample": f"the first {steps} of the 200 control steps (b = 0, mu = {w.mu}): router logits, "
+                      f"softmax + biased top-K + counts and the bias update of T = {w.T} tokens each",
+            "control_step_ms": round(1e3 * step_s, 1), "tokens_per_s": round(w.T / step_s, 1)}
 
 
 def main():
@@ -793,7 +821,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-route-tokens", type=int, default=None,
                     help="tokens the CPU baseline routes (default: the whole batch)")
-    ap.add_argument("--cpu-ffn-tokens", type=int, default=256,
+    ap.add_argument("--cpu-ffn-tokens", type=int, default=512,
                     help="tokens whose FFN picks the CPU baseline runs through the experts")
     ap.add_argument("--ref-tokens", type=int, default=8, help="tokens per reference-arm step")
     ap.add_argument("--experts", choices=["bf16", "fp8"], default="bf16",

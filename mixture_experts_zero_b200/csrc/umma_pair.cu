@@ -157,6 +157,32 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, uint6
 // epilogue three times longer (15 against 5 us per 128 x 128 block), and H is rounded to bf16.
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
+// Row tile store of one warp's 32-row x 32-feature bf16 block, held one row per lane (pk: the
+// lane's 64 bytes). The block goes through the warp's transpose buffer, so that each store
+// instruction writes eight whole 64-byte row segments instead of 32 scattered 16-byte pieces.
+// Rows nv .. 31 are skipped; dst = the block's first output element (row of lane 0); the whole
+// warp calls it.
+__device__ __forceinline__ void store_row_block(uint8_t* xp, const uint32_t (&pk)[16], int nv,
+                                                __nv_bfloat16* dst, int64_t ldo) {
+    const int lane = threadIdx.x & 31;
+    if (lane < nv) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(xp + lane * XPOSE_ROW + (((j ^ (lane >> 1)) & 3) << 4)) =
+                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+    }
+    __syncwarp();
+    const int k = lane & 3;
+#pragma unroll
+    for (int i2 = 0; i2 < 4; ++i2) {
+        const int rr = (lane >> 2) + 8 * i2;
+        if (rr < nv)
+            *reinterpret_cast<uint4*>(dst + rr * ldo + k * 8) =
+                *reinterpret_cast<const uint4*>(xp + rr * XPOSE_ROW + (((k ^ (rr >> 1)) & 3) << 4));
+    }
+    __syncwarp();
+}
+
 template <bool F8>
 __device__ __forceinline__ void mma_step(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t accumulate) {
@@ -483,6 +509,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 const int r = static_cast<int>(rank) * HALF_M + i;  // row within the 256-row tile
                 const int64_t grow = tl.row0 + r;
                 const bool valid = r < tl.rows && grow < g.rows_cap;
+                // the warp's 32 rows start at rb; nv of them are real rows
+                const int rb = static_cast<int>(rank) * HALF_M + q * 32;
+                int64_t nv64 = g.rows_cap - (tl.row0 + rb);
+                if (nv64 > tl.rows - rb) nv64 = tl.rows - rb;
+                const int nv = nv64 < 0 ? 0 : (nv64 > 32 ? 32 : static_cast<int>(nv64));
+                uint8_t* xp = smem + Layout::xpose_off + (warp - EPI_WARP0) * XPOSE_WARP;
+                __nv_bfloat16* out_rb = out + (tl.row0 + rb) * g.ldo;
                 if (MODE == MODE_SWIGLU) {
                     // the next 32 columns' TMEM loads are in flight while this block is computed
                     uint32_t gbuf[2][32], ubuf[2][32];
@@ -499,6 +532,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         uint32_t (&gv)[32] = gbuf[ci & 1];
                         uint32_t (&uv)[32] = ubuf[ci & 1];
                         const int f0 = fbase + c;
+                        uint32_t pk[16];
                         if (valid && f0 < g.n_out) {
                             if (F8) {
                                 // (acc * row scale) * weight-row scale, gate and up separately
@@ -518,16 +552,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                                     }
                                 }
                             }
-                            uint32_t pk[16];
 #pragma unroll
                             for (int j = 0; j < 16; ++j)
                                 pk[j] = pack_bf16x2(silu_mul(__uint_as_float(gv[2 * j]), __uint_as_float(uv[2 * j])),
                                                     silu_mul(__uint_as_float(gv[2 * j + 1]), __uint_as_float(uv[2 * j + 1])));
-                            uint4* d4 = reinterpret_cast<uint4*>(out + grow * g.ldo + f0);
-#pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                d4[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
                         }
+                        if (nv > 0 && f0 < g.n_out) store_row_block(xp, pk, nv, out_rb + f0, g.ldo);
                     }
                 } else {
                     for (int c = 0; c < 2 * HALF_M; c += 32) {
@@ -535,6 +565,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         tmem_ld_32x32b_x32(tb + c, v);
                         tmem_ld_wait();
                         const int f0 = fbase + c;
+                        uint32_t pk[16];
                         if (valid && f0 < g.n_out) {
                             if (F8) {
                                 // (acc * row scale) * weight-row scale
@@ -550,15 +581,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                                         v[4 * j4 + u] = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j4 + u]), sr), sa[u]));
                                 }
                             }
-                            uint32_t pk[16];
 #pragma unroll
                             for (int j = 0; j < 16; ++j)
                                 pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-                            uint4* d4 = reinterpret_cast<uint4*>(out + grow * g.ldo + f0);
-#pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                d4[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
                         }
+                        if (nv > 0 && f0 < g.n_out) store_row_block(xp, pk, nv, out_rb + f0, g.ldo);
                     }
                 }
             } else {
