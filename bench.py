@@ -817,7 +817,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill",
-                    choices=["prefill", "decode", "small", "tiny", "prefill_ncu", "route_ncu", "decode_ncu"])
+                    choices=["prefill", "decode", "small", "tiny", "prefill_ncu", "route_ncu", "decode_ncu",
+                             "cold_ncu"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-route-tokens", type=int, default=None,
                     help="tokens the CPU baseline routes (default: the whole batch)")

@@ -35,6 +35,12 @@
 //   weight tiles ("swap"): 256 weight rows (128 per CTA) on the M side and the rows of one expert,
 //     rounded up to 64 and split between the CTAs, on the N side (N <= 128 for GEMM 1, <= 256 for
 //     GEMM 2). GEMM 1 issues a gate MMA into columns [0, N) and an up MMA into [128, 128 + N).
+//     A GEMM 2 weight tile of N <= 128 is "double" (when d is a multiple of 512): it loads two
+//     boxes of weight rows per k-step, 256 output features apart, and issues their MMAs on the
+//     same token rows into columns [0, N) and [128, 128 + N): 512 features per tile, so a stage
+//     carries twice the weight bytes per token byte and the ring keeps 5/3 the weight bytes in
+//     flight of a plain weight tile (the cold experts' tiles are a weight stream whose rate per
+//     SM is set by the bytes in flight).
 // Accumulators: a wide row tile takes both; every other tile takes the next one in turn, so the
 // epilogue of one weight tile or narrow row tile overlaps the main loop of the next.
 // Per expert with c_e rows: below cold_rows it is "cold" and runs as weight tiles only; otherwise
@@ -70,13 +76,14 @@ enum Mode : int { MODE_SWIGLU = 1, MODE_DOWN = 2 };
 
 // Shared-memory ring of each GEMM. GEMM 1 stages hold the row box and two weight boxes (a wide
 // row tile's two accumulators, or a weight tile's gate and up rows plus up to 64 token rows): 48 KB
-// in 4 stages. GEMM 2 stages hold two boxes (rows and weights, or weights and up to 128 token rows):
-// 32 KB, so the same shared memory holds 6 stages, half again the bytes in flight of the weight
-// stream that the cold experts' tiles are.
+// in 4 stages. GEMM 2 stages hold two boxes (rows and weights, or weights and up to 128 token
+// rows) or a double weight tile's two weight boxes and up to 64 token rows: 40 KB in 5 stages.
+// `stages` is the depth when the per-expert tables fit beside it; launch_pair takes one stage
+// fewer at a time until they do (very many experts).
 template <int MODE>
 struct Ring {
-    static constexpr int stages = MODE == MODE_DOWN ? 6 : 4;
-    static constexpr int bytes = MODE == MODE_DOWN ? 2 * A_BYTES : 3 * A_BYTES;
+    static constexpr int stages = MODE == MODE_DOWN ? 5 : 4;
+    static constexpr int bytes = MODE == MODE_DOWN ? 2 * A_BYTES + 64 * BK * 2 : 3 * A_BYTES;
 };
 
 struct PairArgs {
@@ -98,6 +105,8 @@ struct PairArgs {
     int rem_rows;            // an expert's rows past its last full 256-row tile: fewer than this
                              // run as weight tiles, otherwise as one more row tile
     int wide;                // row tiles span two accumulators (2 * tile_cols output columns)
+    int dbl;                 // GEMM 2: weight tiles of N <= 128 cover 512 output features
+    int stages;              // ring depth (set by launch_pair)
     const float* row_scale;  // E4M3 GEMM 1: scale of each grouped row [rows_cap]
     const float* w_scale;    // E4M3 GEMM 1: scale of each weight row [n_groups * b_group_rows]
     int64_t abort_kstep;     // test switch: the MMA issuer gives up before this k-step (< 0: never)
@@ -109,20 +118,24 @@ struct PairArgs {
 constexpr int XPOSE_ROW = 64;
 constexpr int XPOSE_WARP = 32 * XPOSE_ROW;
 
+// Shared memory of one CTA with a ring of `st` stages: the ring, the barriers (full and empty per
+// stage, tfull[2], tempty[2], drain), the TMEM address and abort flag, the epilogue transpose
+// tiles, the per-expert tile prefix sums.
 template <int MODE>
 struct Layout {
-    static constexpr int STAGES = Ring<MODE>::stages;
-    static constexpr int bars_off = STAGES * Ring<MODE>::bytes;
-    static constexpr int n_bars = 2 * STAGES + 5;  // full, empty, tfull[2], tempty[2], drain
-    static constexpr int misc_off = bars_off + n_bars * 8;
-    static constexpr int xpose_off = (misc_off + 16 + 127) & ~127;
-    static constexpr int table_off = xpose_off + 8 * XPOSE_WARP;
-    static size_t bytes(int n_groups) { return 1024 + table_off + 2 * static_cast<size_t>(n_groups + 1) * 4; }
+    int bars_off, misc_off, xpose_off, table_off;
+    __host__ __device__ explicit Layout(int st)
+        : bars_off(st * Ring<MODE>::bytes),
+          misc_off(bars_off + (2 * st + 5) * 8),
+          xpose_off((misc_off + 16 + 127) & ~127),
+          table_off(xpose_off + 8 * XPOSE_WARP) {}
+    size_t bytes(int n_groups) const { return 1024 + table_off + 2 * static_cast<size_t>(n_groups + 1) * 4; }
 };
 
 struct Tile {
     int swap;
     int wide;  // row tile over both accumulators
+    int dbl;   // double weight tile (GEMM 2, 512 output features)
     int grp;
     int64_t row0;
     int rows;
@@ -207,23 +220,24 @@ template <int MODE, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     umma_pair_kernel(const __grid_constant__ CUtensorMap mapRows, const __grid_constant__ CUtensorMap mapW,
                      const __grid_constant__ CUtensorMap mapTok, const PairArgs g) {
-    constexpr int STAGES = Ring<MODE>::stages;
+    // GEMM 1's depth is fixed (its tables always fit); GEMM 2's is set per launch
+    const int STAGES = MODE == MODE_DOWN ? g.stages : Ring<MODE>::stages;
     constexpr int STAGE_BYTES = Ring<MODE>::bytes;
-    using Layout = ::lcmoe::Layout<MODE>;
+    const Layout<MODE> L(STAGES);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + Layout::bars_off);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars_off);
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Layout::misc_off);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Layout::misc_off + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc_off);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc_off + 4);
     // group row offsets are read from global memory (L1-resident after the first tiles); shared
     // memory holds the per-expert tile prefix sums
     const int32_t* __restrict__ offs = g.offsets;
-    int32_t* rpre_s = reinterpret_cast<int32_t*>(smem + Layout::table_off);
+    int32_t* rpre_s = reinterpret_cast<int32_t*>(smem + L.table_off);
     int32_t* spre_s = rpre_s + (g.n_groups + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -272,12 +286,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     set_status(g.status, LC_MOE_DEV_IDX_RANGE);
                 }
                 if (cnt > 0 && cnt < g.cold_rows) {
-                    nc = g.s_tiles;
+                    nc = (g.dbl && cnt <= HALF_M) ? g.s_tiles / 2 : g.s_tiles;
                 } else if (cnt > 0) {
                     const int nfull = cnt / (2 * HALF_M);
                     const int rem = cnt - nfull * 2 * HALF_M;
                     const bool rem_row = rem >= g.rem_rows;
-                    nh = (nfull + (rem_row ? 1 : 0)) * g.ntiles + ((rem > 0 && !rem_row) ? g.s_tiles : 0);
+                    nh = (nfull + (rem_row ? 1 : 0)) * g.ntiles;
+                    if (rem > 0 && !rem_row) nh += (g.dbl && rem <= HALF_M) ? g.s_tiles / 2 : g.s_tiles;
                 }
             }
             int ih = nh, ic = nc;
@@ -320,6 +335,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const int rem = cnt - nfull * 2 * HALF_M;
             const int nrow = (nfull + (rem >= g.rem_rows ? 1 : 0)) * g.ntiles;
             tl.grp = e;
+            tl.dbl = 0;
             if (local < nrow) {
                 const int mt = local / g.ntiles;
                 tl.swap = 0;
@@ -333,7 +349,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 tl.wide = 0;
                 tl.row0 = static_cast<int64_t>(__ldg(offs + (e))) + static_cast<int64_t>(nfull) * 2 * HALF_M;
                 tl.rows = rem;
-                tl.n0 = (local - nrow) * 2 * HALF_M;
+                tl.dbl = g.dbl && rem <= HALF_M;
+                tl.n0 = (local - nrow) * (tl.dbl ? 4 : 2) * HALF_M;
                 tl.ntok = (rem + TOK_ROUND - 1) / TOK_ROUND * TOK_ROUND;
             }
         } else {
@@ -345,7 +362,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             tl.grp = e;
             tl.row0 = __ldg(offs + (e));
             tl.rows = __ldg(offs + (e + 1)) - __ldg(offs + (e));
-            tl.n0 = (idx - spre_s[e]) * 2 * HALF_M;
+            tl.dbl = g.dbl && tl.rows <= HALF_M;
+            tl.n0 = (idx - spre_s[e]) * (tl.dbl ? 4 : 2) * HALF_M;
             tl.ntok = (tl.rows + TOK_ROUND - 1) / TOK_ROUND * TOK_ROUND;
         }
         return tl;
@@ -364,7 +382,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const int tok_rows = tl.ntok / 2;  // this CTA's share of the N side
             uint32_t cta_bytes;
             if (!tl.swap) cta_bytes = (tl.wide ? 3 : 2) * A_BYTES;
-            else cta_bytes = (MODE == MODE_SWIGLU ? 2 : 1) * A_BYTES + tok_rows * BK * 2;
+            else cta_bytes = ((MODE == MODE_SWIGLU || tl.dbl) ? 2 : 1) * A_BYTES + tok_rows * BK * 2;
             const int wbase = tl.grp * g.b_group_rows;
             for (int kb = 0; kb < nk; ++kb) {
                 if (!mbar_wait(&empty[s], ph ^ 1u, g.wait_ns, abort_flag, g.status)) {
@@ -389,8 +407,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     const int wrow = wbase + tl.n0 + static_cast<int>(rank) * HALF_M;
                     tma_load_2d_pair(sa, &mapW, bar, kx, wrow, pol_stream);
                     uint8_t* st = sb;
-                    if (MODE == MODE_SWIGLU) {
-                        tma_load_2d_pair(sb, &mapW, bar, kx, wrow + g.up_off, pol_stream);
+                    if (MODE == MODE_SWIGLU || tl.dbl) {
+                        // GEMM 1: the up rows of the same features; double tile: the weight rows
+                        // 256 features further on
+                        tma_load_2d_pair(sb, &mapW, bar, kx, wrow + (MODE == MODE_SWIGLU ? g.up_off : 2 * HALF_M),
+                                         pol_stream);
                         st = sb + A_BYTES;
                     }
                     const int64_t t0 = tl.row0 + static_cast<int64_t>(rank) * tok_rows;
@@ -449,7 +470,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 const uint8_t* sa = smem + s * STAGE_BYTES;
                 const uint64_t ad = sw128_kmajor_desc(smem_u32(sa));
                 const uint64_t bd = sw128_kmajor_desc(smem_u32(sa + A_BYTES));
-                if (MODE == MODE_SWIGLU && tl.swap) {
+                if (tl.swap && (MODE == MODE_SWIGLU || tl.dbl)) {
                     const uint64_t td = sw128_kmajor_desc(smem_u32(sa + 2 * A_BYTES));
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
@@ -514,7 +535,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 int64_t nv64 = g.rows_cap - (tl.row0 + rb);
                 if (nv64 > tl.rows - rb) nv64 = tl.rows - rb;
                 const int nv = nv64 < 0 ? 0 : (nv64 > 32 ? 32 : static_cast<int>(nv64));
-                uint8_t* xp = smem + Layout::xpose_off + (warp - EPI_WARP0) * XPOSE_WARP;
+                uint8_t* xp = smem + L.xpose_off + (warp - EPI_WARP0) * XPOSE_WARP;
                 __nv_bfloat16* out_rb = out + (tl.row0 + rb) * g.ldo;
                 if (MODE == MODE_SWIGLU) {
                     // the next 32 columns' TMEM loads are in flight while this block is computed
@@ -592,14 +613,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 // weight tile: lane = output feature, column = row of the expert's group. Each
                 // 32 x 32 block goes through shared memory transposed, so that every thread then
                 // stores 32 consecutive features of one row as four 16-byte vectors.
-                uint8_t* xp = smem + Layout::xpose_off + (warp - EPI_WARP0) * XPOSE_WARP;
-                const int f0 = tl.n0 + static_cast<int>(rank) * HALF_M + q * 32;  // warp's first feature
+                // A double weight tile's second 256 features are in columns [128, 128 + N).
+                uint8_t* xp = smem + L.xpose_off + (warp - EPI_WARP0) * XPOSE_WARP;
+                for (int half = 0; half < ((MODE == MODE_DOWN && tl.dbl) ? 2 : 1); ++half) {
+                const int f0 = tl.n0 + half * 2 * HALF_M + static_cast<int>(rank) * HALF_M + q * 32;  // warp's first feature
+                const uint32_t tbh = tb + static_cast<uint32_t>(half * HALF_M);
                 for (int c0 = 0; c0 < tl.ntok; c0 += 32) {
                     uint32_t v[32];
-                    tmem_ld_32x32b_x32(tb + c0, v);
+                    tmem_ld_32x32b_x32(tbh + c0, v);
                     if (MODE == MODE_SWIGLU) {
                         uint32_t uv[32];
-                        tmem_ld_32x32b_x32(tb + HALF_M + c0, uv);
+                        tmem_ld_32x32b_x32(tbh + HALF_M + c0, uv);
                         tmem_ld_wait();
                         if (F8) {
                             // lane = weight row (feature), column j = grouped row c0 + j
@@ -650,6 +674,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     }
                     __syncwarp();
                 }
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -671,7 +696,7 @@ cudaError_t launch_pair(const CUtensorMap& mr, const CUtensorMap& mw, const CUte
                         const PairArgs& args, int grid, cudaStream_t st) {
     // a GEMM 2 stage holds two boxes: its row tiles are never wide
     if (MODE == MODE_DOWN && args.wide) return cudaErrorInvalidValue;
-    const size_t smem = Layout<MODE>::bytes(args.n_groups);
+    if (MODE == MODE_SWIGLU && args.dbl) return cudaErrorInvalidValue;
     // once per device: allow the kernel the device's whole opt-in shared memory
     static PerDeviceOnce setup;
     static int max_optin[PerDeviceOnce::kMaxDevices];
@@ -686,8 +711,14 @@ cudaError_t launch_pair(const CUtensorMap& mr, const CUtensorMap& mw, const CUte
     if (e != cudaSuccess) return e;
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    // the ring as deep as the per-expert tables leave room for (at least two stages)
+    PairArgs a = args;
+    a.stages = Ring<MODE>::stages;
+    if (MODE == MODE_DOWN)
+        while (a.stages > 2 && Layout<MODE>(a.stages).bytes(a.n_groups) > static_cast<size_t>(max_optin[dev])) --a.stages;
+    const size_t smem = Layout<MODE>(a.stages).bytes(a.n_groups);
     if (smem > static_cast<size_t>(max_optin[dev])) return cudaErrorInvalidValue;
-    umma_pair_kernel<MODE, F8><<<grid, NUM_THREADS, smem, st>>>(mr, mw, mt, args);
+    umma_pair_kernel<MODE, F8><<<grid, NUM_THREADS, smem, st>>>(mr, mw, mt, a);
     return cudaGetLastError();
 }
 
@@ -793,6 +824,7 @@ PairArgs down_args(int64_t rows_cap, const int32_t* offsets, int N, int d, int I
     a.s_tiles = (d + 2 * HALF_M - 1) / (2 * HALF_M);
     a.cold_rows = 256;
     a.rem_rows = 256;
+    a.dbl = d % (4 * HALF_M) == 0 ? 1 : 0;
     return a;
 }
 

@@ -64,6 +64,10 @@ WORKLOADS = {
     # LongCat-Flash router shape at decode batch size (T = 128) with 64-wide experts (~0.8 GB on
     # the device): profiler captures of the small-batch routing and one-launch grouping
     "decode_ncu": Workload("decode_ncu", T=128, d=6144, N=512, Z=256, K=12, K_e=8, I=64, seed=2),
+    # LongCat-Flash expert shape with 64 FFN + 32 zero experts and 512 tokens (~64 rows per FFN
+    # expert, so every expert is cold: weight tiles only; ~4.9 GB on the device): profiler captures
+    # of the expert GEMMs as weight streams
+    "cold_ncu": Workload("cold_ncu", T=512, d=6144, N=64, Z=32, K=12, K_e=8, I=2048, seed=2),
     # bias-control loop: 200 fresh batches of 8192 tokens, routing only
     "bias_loop": Workload("bias_loop", T=8192, d=6144, N=512, Z=256, K=12, K_e=8, I=2048,
                           seed=4, steps=200),
