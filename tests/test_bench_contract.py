@@ -73,3 +73,31 @@ def test_cpu_baseline_batches_the_expert_rows_and_names_its_phases():
     assert "subset-measured" in cb["sample"] and f"{cb['cores']} threads" in cb["sample"]
     # N = 8 experts in groups of 4: two oracle calls, each with the rows of four experts
     assert "2 oracle calls" in cb["sample"]
+
+
+def test_cpu_baseline_of_a_whole_batch_says_so():
+    """With the FFN sample as large as the batch, every token is routed and run through the
+    experts: the line is labelled a full-batch measurement."""
+    sys.path.insert(0, str(ROOT))
+    import bench
+    from mixture_experts_zero_b200 import inputs
+    w = inputs.WORKLOADS["tiny"]
+    cb = bench.cpu_baseline(w, inputs.make(w, device="cpu"), ffn_tokens=w.T)
+    assert cb["tokens"]["routed"] == w.T and cb["tokens"]["ffn"] == w.T
+    assert cb["sample"].startswith("full batch: ")
+
+
+def test_control_loop_cpu_baseline_times_route_and_update():
+    """The bias-control loop's CPU baseline: the oracle's router logits, routing and bias update
+    on the loop's first steps, reported per control step and per token."""
+    sys.path.insert(0, str(ROOT))
+    import bench
+    import oracle
+    from mixture_experts_zero_b200 import inputs
+    w = inputs.scaled(inputs.WORKLOADS["bias_loop"], T=64, d=256)
+    line = bench.control_cpu_baseline(w, "cpu", steps=2)
+    assert line["impl"] == "cpu_baseline" and line["kind"] == "oracle"
+    assert line["cores"] == oracle.num_threads()
+    assert line["control_step_ms"] > 0
+    assert abs(line["tokens_per_s"] - w.T / (line["control_step_ms"] / 1e3)) <= 0.01 * line["tokens_per_s"] + 1
+    assert "first 2 of the 200 control steps" in line["sample"]
