@@ -807,7 +807,7 @@ def control_cpu_baseline(w, dev, steps: int = 2):
             "cpu": cpu_model(), "host_cpus": os.cpu_count(),
             "sample": f"the first {steps} of the {w.steps} control steps (b = 0, mu = {w.mu}): router logits, "
                       f"softmax + biased top-K + counts and the bias update of T = {w.T} tokens each",
-            "control_step_ms": round(1e3 * step_s, 1), "tokens_per_s": round(w.T / step_s, 1)}
+            "control_step_ms": round(1e3 * step_s, 3), "tokens_per_s": round(w.T / step_s, 1)}
 
 
 def main():

@@ -99,5 +99,7 @@ def test_control_loop_cpu_baseline_times_route_and_update():
     assert line["impl"] == "cpu_baseline" and line["kind"] == "oracle"
     assert line["cores"] == oracle.num_threads()
     assert line["control_step_ms"] > 0
-    assert abs(line["tokens_per_s"] - w.T / (line["control_step_ms"] / 1e3)) <= 0.01 * line["tokens_per_s"] + 1
+    # both figures come from the same mean step time (the milliseconds rounded to 1 us)
+    ms = line["control_step_ms"]
+    assert abs(line["tokens_per_s"] - w.T / (ms / 1e3)) <= (0.0005 / ms + 1e-6) * line["tokens_per_s"] + 0.1
     assert "first 2 of the 200 control steps" in line["sample"]
