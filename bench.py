@@ -157,6 +157,44 @@ def traffic_record(key: str):
     return rec
 
 
+def gemm_phase_roofline(counts, d: int, I: int, f8: bool, mhz: dict, sm_count: int, hbm_gbs: float,
+                        measured_ms: dict) -> dict:
+    """Each expert GEMM split by the kind of tile its rows take: rows in 256-row tiles are tensor
+    work at the SM clock measured inside the kernel (8192 bf16 / 16384 E4M3 FLOP per SM per
+    cycle), the other rows' experts (cold experts, and the leftover rows of hot ones) are weight
+    streams at the measured copy bandwidth; the bound runs the two kinds one after the other.
+    GEMM 1 (gate/up): row tiles from 128 rows (a 128..255-row remainder included); GEMM 2: from
+    256. counts: rows per FFN expert."""
+    out = {}
+    wb = 1 if f8 else 2
+    for name, cold, rem_rows, fl_per_row, w_bytes in (
+            ("gemm1_swiglu", 128, 128, 4.0 * d * I, 2 * I * d * wb),
+            ("gemm2_down", 256, 256, 2.0 * d * I, d * I * wb)):
+        if not mhz.get(name):
+            continue
+        hot_rows = 0
+        stream_bytes = 0
+        for n in counts:
+            n = int(n)
+            if n == 0:
+                continue
+            if n < cold:
+                stream_bytes += w_bytes
+                continue
+            nfull, rem = divmod(n, 256)
+            hot_rows += nfull * 256 + (rem if rem >= rem_rows else 0)
+            if 0 < rem < rem_rows:
+                stream_bytes += w_bytes
+        rate = sm_count * (16384 if f8 else 8192) * mhz[name] * 1e6
+        t_hot = fl_per_row * hot_rows / rate
+        t_stream = stream_bytes / (hbm_gbs * 1e9)
+        out[name] = {"t_bound_ms": round((t_hot + t_stream) * 1e3, 4),
+                     "frac": round((t_hot + t_stream) * 1e3 / measured_ms[name], 4),
+                     "tensor_ms": round(t_hot * 1e3, 4), "stream_ms": round(t_stream * 1e3, 4),
+                     "rows_in_row_tiles": hot_rows, "weight_stream_bytes": stream_bytes}
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -233,6 +271,10 @@ def run_ours(args):
         pass
     sampler = ClockSampler(uuid)
     sampler.start()
+    # the grouped GEMMs stamp the global timer and their SM's cycle counter at the start and end
+    # of CTA 0 (the last timed step's launches remain): the SM clock inside each GEMM
+    probe = torch.zeros(8, dtype=torch.int64, device=dev)
+    B.lc_moe_set_clock_probe(probe)
     time.sleep(0.3)
     barrier()
     t_start.record(stream)
@@ -240,7 +282,12 @@ def run_ours(args):
         step(events=ev[i])
     t_end.record(stream)
     barrier()
+    B.lc_moe_set_clock_probe(None)
     clock_rows = sampler.stop()
+    pr = probe.cpu().tolist()
+    gemm_mhz = {name: (round((pr[o + 3] - pr[o + 1]) / (pr[o + 2] - pr[o]) * 1e3, 1) if pr[o + 2] > pr[o] else None)
+                for name, o in (("gemm1_swiglu", 0), ("gemm2_down", 4))}
+    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
     elapsed_ms = t_start.elapsed_time(t_end)
     stage_ms = np.array([[row[j].elapsed_time(row[j + 1]) for j in range(len(STAGES))] for row in ev])
     if B.lc_moe_read_status(ws, stream=stream, raise_on_error=False):
@@ -350,6 +397,12 @@ def run_ours(args):
                         "share": round(float(mean[j] / mean.sum()), 4), "bound": bound,
                         "achieved": round(ach, 2), "unit": unit, "peak": peak,
                         "frac": round(ach / peak, 4), "algorithmic_work": work}
+        if gemm_mhz.get(name):
+            # the nominal dense tensor rate at the clock measured inside the kernel: 8192 bf16
+            # (16384 E4M3) FLOP per SM per cycle
+            rate = sm_count * (16384 if f8 else 8192) * gemm_mhz[name] * 1e6 / 1e12
+            stages[name]["sm_mhz_in_kernel"] = gemm_mhz[name]
+            stages[name]["frac_of_tensor_rate_at_that_clock"] = round(ach / rate, 4)
     dom = max(STAGES, key=lambda n: stages[n]["ms"])
     ds = stages[dom]
     trec = traffic_record(f"{w.name}/{dom}" + ("@fp8" if f8 else ""))
@@ -362,6 +415,11 @@ def run_ours(args):
                                 + ", MEASURED_PEAKS.json)") if peak_src == "measured" else "fallback",
                 "traffic": (trec["dram_bytes_per_launch"] if trec else None),
                 "algorithmic_per_launch": ds["algorithmic_work"]}
+    if "sm_mhz_in_kernel" in ds:
+        roofline["sm_mhz_in_kernel"] = ds["sm_mhz_in_kernel"]
+        roofline["frac_of_tensor_rate_at_that_clock"] = ds["frac_of_tensor_rate_at_that_clock"]
+    phase_roofline = gemm_phase_roofline(c[: w.N], d_, I_, f8, gemm_mhz, sm_count, peaks["hbm_gbs"],
+                                         {n: stages[n]["ms"] for n in ("gemm1_swiglu", "gemm2_down")})
     # whole-step roofline: max(FLOP / sustained TC peak, touched weights + activations / HBM)
     flops = 2.0 * T * d_ * E + 6.0 * M * d_ * I_
     bytes_ = wbytes_touched + E * d_ * 2 + 2 * T * d_ * 2
@@ -384,6 +442,7 @@ def run_ours(args):
                                f"[{lo},{hi})": int(((c[:w.N] >= lo) & (c[:w.N] < hi)).sum())
                                for lo, hi in ((1, 128), (128, 256), (256, 512), (512, 1024), (1024, T + 1))}},
         "stages": stages,
+        "gemm_phase_roofline": phase_roofline,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": int(x.numel() * 2),
                 "d2h_bytes_per_step": int(out.numel() * 2), "steps": e2e_steps_n,
                 "copies": "pinned host x -> device and out -> pinned host every step, on a copy "

@@ -111,6 +111,15 @@ size_t lc_moe_workspace_bytes(const lc_moe_shape* s, int op);
  * returns early with partial results. Values below 1e6 are raised to 1e6. */
 void lc_moe_set_wait_limit_ns(uint64_t limit_ns);
 
+/* Clock probe of the grouped expert GEMMs, for measurement. While set, every launch of grouped
+ * GEMM 1 (gate/up + SwiGLU) writes, from the first thread of its CTA 0, the global timer (ns) and
+ * that SM's cycle counter when the CTA starts its tiles and when it has finished them, to
+ * probe[0..3] (start ns, start cycles, end ns, end cycles); grouped GEMM 2 writes probe[4..7].
+ * (end cycles - start cycles) / (end ns - start ns) is the SM clock the launch ran at. probe:
+ * device memory of 8 uint64 (the caller's, 8-byte aligned), or NULL to stop (the default).
+ * Process-wide like the wait limit; each launch overwrites its four values. */
+void lc_moe_set_clock_probe(void* probe);
+
 /* Device check of the bounded waits: one CTA runs the pipelines' bounded wait on a barrier phase
  * that nothing completes (role 0, the current limit) and on the phase role 0 would have released
  * (role 1, four times the limit). On a working device role 0 gives up after the limit, sets

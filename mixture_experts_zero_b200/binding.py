@@ -31,7 +31,7 @@ EXPORTED = (
     "lc_moe_read_status", "lc_moe_router_logits", "lc_moe_topk", "lc_moe_expert_hist",
     "lc_moe_permute", "lc_moe_expert_ffn", "lc_moe_combine", "lc_moe_permute_noalloc",
     "lc_moe_quantize_e4m3", "lc_moe_forward_fp8", "lc_moe_forward_fp8_timed",
-    "lc_moe_check_wait_timeout", "lc_moe_ep_regroup_plan", "lc_moe_copy_rows",
+    "lc_moe_check_wait_timeout", "lc_moe_ep_regroup_plan", "lc_moe_copy_rows", "lc_moe_set_clock_probe",
 )
 
 
@@ -73,6 +73,8 @@ def _configure(L: ctypes.CDLL) -> ctypes.CDLL:
     L.lc_moe_workspace_bytes.restype = SZ
     L.lc_moe_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     L.lc_moe_set_wait_limit_ns.restype = None
+    L.lc_moe_set_clock_probe.argtypes = [P]
+    L.lc_moe_set_clock_probe.restype = None
     fwd = [SP, P, P, P, P, P, P, P, P, P, P, SZ, P]
     L.lc_moe_forward.argtypes = fwd
     L.lc_moe_forward_timed.argtypes = fwd + [ctypes.POINTER(P)]
@@ -145,6 +147,14 @@ def new_workspace(shape: Shape, op: int = OP_FORWARD, device=None) -> torch.Tens
 
 def lc_moe_set_wait_limit_ns(limit_ns: int) -> None:
     _lib().lc_moe_set_wait_limit_ns(int(limit_ns))
+
+
+def lc_moe_set_clock_probe(probe) -> None:
+    """probe: int64 device tensor of 8 elements (GEMM 1: start ns, start cycles, end ns, end
+    cycles of CTA 0; GEMM 2 the same), or None to stop."""
+    if probe is not None:
+        assert probe.is_cuda and probe.dtype == torch.int64 and probe.numel() >= 8 and probe.is_contiguous()
+    _lib().lc_moe_set_clock_probe(None if probe is None else _ptr(probe))
 
 
 def _dims(x, wr, w13=None, w2=None, K=None):

@@ -13,6 +13,7 @@ namespace lcmoe {
 namespace {
 
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+std::atomic<unsigned long long*> g_clock_probe{nullptr};
 
 constexpr size_t kAlign = 256;
 constexpr size_t kStatusBytes = 256;
@@ -206,6 +207,8 @@ const DevInfo* current_device_info() {
 
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
+unsigned long long* clock_probe() { return g_clock_probe.load(std::memory_order_relaxed); }
+
 }  // namespace lcmoe
 
 using namespace lcmoe;
@@ -244,6 +247,10 @@ size_t lc_moe_workspace_bytes(const lc_moe_shape* s, int op) {
 void lc_moe_set_wait_limit_ns(uint64_t limit_ns) {
     if (limit_ns < 1000000ull) limit_ns = 1000000ull;
     g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+}
+
+void lc_moe_set_clock_probe(void* probe) {
+    g_clock_probe.store(static_cast<unsigned long long*>(probe), std::memory_order_relaxed);
 }
 
 int lc_moe_check_wait_timeout(void* ws, size_t ws_bytes, void* stream) {

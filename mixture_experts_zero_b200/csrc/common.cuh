@@ -367,6 +367,8 @@ class PerDeviceOnce {
 const DevInfo* current_device_info();
 
 uint64_t wait_limit_ns();
+// Device buffer of the grouped GEMMs' clock probe (lc_moe_set_clock_probe), or nullptr.
+unsigned long long* clock_probe();
 
 // Row-major bf16 matrix [rows, cols] as a TMA map with 64 x box_rows boxes and the 128-byte swizzle.
 bool make_tma_map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows);

@@ -110,6 +110,7 @@ struct PairArgs {
     const float* row_scale;  // E4M3 GEMM 1: scale of each grouped row [rows_cap]
     const float* w_scale;    // E4M3 GEMM 1: scale of each weight row [n_groups * b_group_rows]
     int64_t abort_kstep;     // test switch: the MMA issuer gives up before this k-step (< 0: never)
+    unsigned long long* clock_probe;  // [4] start ns, start cycles, end ns, end cycles of CTA 0
 };
 
 // Epilogue transpose tile of one warp: 32 rows x 32 features (bf16), 64 bytes per row, its four
@@ -317,6 +318,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     cluster_sync_all();  // both CTAs' barriers are initialised before any cross-CTA signal
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    if (g.clock_probe && blockIdx.x == 0 && threadIdx.x == 0) {
+        g.clock_probe[0] = globaltimer_ns();
+        g.clock_probe[1] = clock64();
+    }
 
     const int total_r = rpre_s[g.n_groups];
     const int total_s = spre_s[g.n_groups];
@@ -685,6 +690,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 
     __syncthreads();
     cluster_sync_all();  // the leader's MMAs have finished reading the peer's shared memory
+    if (g.clock_probe && blockIdx.x == 0 && threadIdx.x == 0) {
+        g.clock_probe[2] = globaltimer_ns();
+        g.clock_probe[3] = clock64();
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, TMEM_COLS);
@@ -747,6 +756,7 @@ PairArgs swiglu_args(int64_t rows_cap, const int32_t* offsets, int N, int d, int
     a.out = static_cast<__nv_bfloat16*>(h);
     a.status = status;
     a.wait_ns = wait_limit_ns();
+    a.clock_probe = clock_probe();
     a.abort_kstep = debug_abort_kstep();
     a.rows_cap = rows_cap;
     a.ldo = I;
@@ -807,6 +817,7 @@ PairArgs down_args(int64_t rows_cap, const int32_t* offsets, int N, int d, int I
     a.out = static_cast<__nv_bfloat16*>(y);
     a.status = status;
     a.wait_ns = wait_limit_ns();
+    a.clock_probe = clock_probe() ? clock_probe() + 4 : nullptr;
     a.abort_kstep = debug_abort_kstep();
     a.rows_cap = rows_cap;
     a.ldo = d;

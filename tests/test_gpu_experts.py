@@ -114,3 +114,29 @@ def test_combine_matches_oracle(cuda_device, name):
     assert_out_close(got, exact, what="combine")
     # fp32 accumulation vs double: equal after bf16 rounding except near rounding boundaries
     assert assert_within_ulp(got, ref, what="combine") > 0.97
+
+
+def test_clock_probe_reports_each_gemms_sm_clock(cuda_device):
+    """With the clock probe set, each grouped GEMM launch records CTA 0's start and end (global
+    timer and cycle counter); the ratio is a plausible SM clock, and unsetting the probe stops the
+    writes."""
+    d = make("small")
+    w = d["w"]
+    idx, _ = B.lc_moe_route(d["x"], d["wr"], d["bias"], w.K, w.N)
+    offsets, _, _, x_perm = B.lc_moe_permute(idx, w.N, w.E, x=d["x"])
+    probe = torch.zeros(8, dtype=torch.int64, device="cuda")
+    B.lc_moe_set_clock_probe(probe)
+    try:
+        B.lc_moe_expert_ffn(x_perm, offsets, d["w13"], d["w2"], w.T, w.K)
+        torch.cuda.synchronize()
+    finally:
+        B.lc_moe_set_clock_probe(None)
+    p = probe.cpu().tolist()
+    for o in (0, 4):
+        assert p[o + 2] > p[o] > 0 and p[o + 3] > p[o + 1]
+        mhz = (p[o + 3] - p[o + 1]) / (p[o + 2] - p[o]) * 1e3
+        assert 300.0 < mhz < 2500.0, mhz
+    probe.zero_()
+    B.lc_moe_expert_ffn(x_perm, offsets, d["w13"], d["w2"], w.T, w.K)
+    torch.cuda.synchronize()
+    assert int(probe.abs().sum()) == 0
