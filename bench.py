@@ -76,7 +76,8 @@ def load_peaks():
 class ClockSampler:
     FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "enforced.power.limit")
 
     def __init__(self, uuid: str | None):
         self.uuid = uuid
@@ -133,8 +134,10 @@ class ClockSampler:
             for name, v in zip(names, r[6:10]):
                 if v.lower().startswith("active"):
                     reasons.add(name)
+        limits = [num(r[10]) for r in rows if len(r) > 10]
         return {"sm_mhz": float(np.nanmedian(sm[loaded])) if loaded.any() else float(np.nanmedian(sm)),
                 "sm_max_mhz": float(np.nanmax([num(r[3]) for r in rows])),
+                "power_limit_w": float(np.nanmax(limits)) if limits else None,
                 "power_w": float(np.nanmedian(power[loaded])) if loaded.any() else None,
                 "reasons": sorted(reasons), "samples": int(len(rows)),
                 "samples_under_load": int(loaded.sum())}
@@ -456,7 +459,10 @@ def run_ours(args):
         "gpu_launches_note": "kernels of this library inside the device-timed region: "
                              f"{n_kernels + (2 if f8 else 0)} per forward "
                              f"{'(incl. the token-row and H-row quantisers) ' if f8 else ''}+ 1 bias update, per step",
-        "clocks": ClockSampler.summarize(clock_rows),
+        "clocks": dict(ClockSampler.summarize(clock_rows),
+                       sm_mhz_in_gemms={k: v for k, v in gemm_mhz.items() if v},
+                       sm_mhz_in_gemms_note="SM clock inside each expert GEMM of the last timed step, "
+                                            "from the kernels' clock probe (cycles / global-timer ns)"),
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline and not f8:
         result["cpu_baseline"] = cpu_baseline(w, data, route_tokens=args.cpu_route_tokens,
