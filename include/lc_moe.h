@@ -90,7 +90,7 @@ enum {
 enum {
     LC_MOE_STAGE_ROUTER_GEMM = 0,  /* router logits, tensor cores */
     LC_MOE_STAGE_TOPK = 1,         /* softmax + biased top-K + expert histogram */
-    LC_MOE_STAGE_PERMUTE = 2,      /* counting sort of FFN picks by expert (3 kernels) */
+    LC_MOE_STAGE_PERMUTE = 2,      /* counting sort of FFN picks by expert (3 kernels; 1 when T <= 256) */
     LC_MOE_STAGE_GATHER = 3,       /* copy of token rows into expert order */
     LC_MOE_STAGE_GEMM1 = 4,        /* grouped gate/up GEMM with the SwiGLU epilogue */
     LC_MOE_STAGE_GEMM2 = 5,        /* grouped down GEMM */
