@@ -7,7 +7,8 @@ LongCat-Flash-shape prefill batch (T=16384 tokens per GPU, d=6144, 512 FFN exper
 256 zero experts, K=12, K_e=8, Zipf(1.1) expert popularity), synthetic data.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-    python bench.py --sweep ffn_rows|hist      (kernel sweeps, one JSON line per case)
+                    [--workload prefill|decode|small|tiny|...] [--experts bf16|fp8]
+    python bench.py --sweep ffn_rows|hist|ffn_subset|control   (one JSON line per case)
 
 Prints one JSON line (rank 0). ``--impl reference`` times the CPU oracle (test infrastructure) on a
 bounded sample of the same workload instead.
