@@ -30,7 +30,9 @@
  *     allocates and frees no device or pinned memory.
  *   - `ws` must be zero-filled before its first use. Its first 256 bytes hold the device status
  *     word: kernels OR LC_MOE_DEV_* bits into it instead of trapping, and it stays set until
- *     lc_moe_read_status clears it. Calls that share a workspace must be ordered on one stream.
+ *     lc_moe_read_status clears it. The same 256 bytes hold the grouped expert GEMMs' tile
+ *     counters (bytes 64 and 128), which each GEMM launch zeroes on the stream before it runs.
+ *     Calls that share a workspace must be ordered on one stream.
  *   - Host-side checks run before any launch; a failing check returns a status code and
  *     enqueues nothing. Functions never abort, throw or print.
  *   - Every entry point except lc_moe_read_status can be captured in a CUDA graph once it has

@@ -48,8 +48,15 @@
 // at least rem_rows of them, else as weight tiles (N rounded up to 64). GEMM 1: cold_rows =
 // rem_rows = 128; GEMM 2: cold_rows = rem_rows = 256. The tile list (built on the device from
 // offsets, identically by every CTA) is: for each hot expert in order, its row tiles then its
-// leftover weight tiles; then the weight tiles of every cold expert. Tile t goes to cluster
-// t mod (gridDim / 2).
+// leftover weight tiles; then the weight tiles of every cold expert.
+// Tiles are handed out in list order as pairs become free: the leader's producer takes the next
+// tile index from a counter in global memory (zeroed before each launch) when it starts a tile,
+// and passes it to every role of both CTAs through a queue of TQ tile indices in shared memory
+// (a full barrier per slot in each CTA, released by the leader's producer; an empty barrier per
+// slot in the leader, which counts the 18 other readers: the MMA issuer, the eight epilogue warps
+// of each CTA and the peer's producer). The tiles that share a hot expert's weights then start
+// within microseconds of one another, so those weights are read from L2 rather than fetched again,
+// and the pairs finish together. The index past the last tile ends every role's loop.
 // Every wait is bounded (lc_moe_set_wait_limit_ns); a wait that runs out raises a CTA-wide abort,
 // records LC_MOE_DEV_WAIT_TIMEOUT, drains in-flight copies and MMAs, and frees TMEM.
 #include <cudaTypedefs.h>
@@ -71,6 +78,7 @@ constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;              // warps 4..11: two epilogue groups of four warps
 constexpr int TOK_BOX = 32;                 // token rows per TMA box of a weight tile (per CTA)
 constexpr int TOK_ROUND = 2 * TOK_BOX;      // weight-tile N is a multiple of this
+constexpr int TQ = 8;                       // depth of the tile-index queue
 
 enum Mode : int { MODE_SWIGLU = 1, MODE_DOWN = 2 };
 
@@ -111,6 +119,7 @@ struct PairArgs {
     const float* w_scale;    // E4M3 GEMM 1: scale of each weight row [n_groups * b_group_rows]
     int64_t abort_kstep;     // test switch: the MMA issuer gives up before this k-step (< 0: never)
     unsigned long long* clock_probe;  // [4] start ns, start cycles, end ns, end cycles of CTA 0
+    int* tile_ctr;           // next tile index (zeroed before each launch; in the status area)
 };
 
 // Epilogue transpose tile of one warp: 32 rows x 32 features (bf16), 64 bytes per row, its four
@@ -120,15 +129,15 @@ constexpr int XPOSE_ROW = 64;
 constexpr int XPOSE_WARP = 32 * XPOSE_ROW;
 
 // Shared memory of one CTA with a ring of `st` stages: the ring, the barriers (full and empty per
-// stage, tfull[2], tempty[2], drain), the TMEM address and abort flag, the epilogue transpose
-// tiles, the per-expert tile prefix sums.
+// stage, tfull[2], tempty[2], drain), the TMEM address and abort flag, the tile-index queue (full
+// and empty barriers, TQ indices), the epilogue transpose tiles, the per-expert tile prefix sums.
 template <int MODE>
 struct Layout {
     int bars_off, misc_off, xpose_off, table_off;
     __host__ __device__ explicit Layout(int st)
         : bars_off(st * Ring<MODE>::bytes),
           misc_off(bars_off + (2 * st + 5) * 8),
-          xpose_off((misc_off + 16 + 127) & ~127),
+          xpose_off((misc_off + 16 + 2 * TQ * 8 + TQ * 4 + 127) & ~127),
           table_off(xpose_off + 8 * XPOSE_WARP) {}
     size_t bytes(int n_groups) const { return 1024 + table_off + 2 * static_cast<size_t>(n_groups + 1) * 4; }
 };
@@ -235,6 +244,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     uint64_t* drain = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc_off);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc_off + 4);
+    // tile-index queue (see the header comment)
+    uint64_t* tq_full = reinterpret_cast<uint64_t*>(smem + L.misc_off + 16);
+    uint64_t* tq_empty = tq_full + TQ;
+    int* tq = reinterpret_cast<int*>(tq_empty + TQ);
     // group row offsets are read from global memory (L1-resident after the first tiles); shared
     // memory holds the per-expert tile prefix sums
     const int32_t* __restrict__ offs = g.offsets;
@@ -245,8 +258,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
-    const int cluster = blockIdx.x >> 1;
-    const int n_clusters = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -258,6 +269,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             mbar_init(&tempty[a], 8);  // 4 epilogue warps in each CTA of the pair
         }
         mbar_init(drain, 1);
+        for (int i = 0; i < TQ; ++i) {
+            mbar_init(&tq_full[i], 1);
+            mbar_init(&tq_empty[i], 18);
+        }
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&mapRows);
@@ -382,7 +397,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         uint32_t ph = 0;
         int issued = 0;
         bool ok = true;
-        for (int tile = cluster; tile < total && ok; tile += n_clusters) {
+        int nxt = leader ? atomicAdd(g.tile_ctr, 1) : 0;
+        for (int qi = 0; ok; ++qi) {
+            const int slot = qi % TQ;
+            const uint32_t par = (qi / TQ) & 1;
+            int tile;
+            if (leader) {
+                if (qi >= TQ && !mbar_wait_cluster(&tq_empty[slot], par ^ 1u, g.wait_ns, abort_flag, g.status)) {
+                    ok = false;
+                    break;
+                }
+                tile = nxt < total ? nxt : total;
+                tq[slot] = tile;
+                st_shared_cluster_u32(mapa_shared(smem_u32(&tq[slot]), 1), static_cast<uint32_t>(tile));
+                mbar_arrive(&tq_full[slot]);
+                mbar_arrive_cluster(mapa_shared(smem_u32(&tq_full[slot]), 1));
+                if (tile < total) nxt = atomicAdd(g.tile_ctr, 1);
+            } else {
+                if (!mbar_wait_cluster(&tq_full[slot], par, g.wait_ns, abort_flag, g.status)) {
+                    ok = false;
+                    break;
+                }
+                tile = tq[slot];
+                mbar_arrive_cluster(mapa_shared(smem_u32(&tq_empty[slot]), 0));
+            }
+            if (tile >= total) break;
             const Tile tl = decode(tile);
             const int tok_rows = tl.ntok / 2;  // this CTA's share of the N side
             uint32_t cta_bytes;
@@ -448,7 +487,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         AccSchedule sched;
         bool ok = true;
         int64_t ksteps = 0;
-        for (int tile = cluster; tile < total && ok; tile += n_clusters) {
+        for (int qi = 0; ok; ++qi) {
+            const int slot = qi % TQ;
+            if (!mbar_wait(&tq_full[slot], (qi / TQ) & 1, g.wait_ns, abort_flag, g.status)) break;
+            const int tile = tq[slot];
+            mbar_arrive(&tq_empty[slot]);
+            if (tile >= total) break;
             const Tile tl = decode(tile);
             const uint32_t idesc = F8 ? idesc_e4m3_f32(2 * HALF_M, tl.swap ? tl.ntok : 2 * HALF_M)
                                       : idesc_bf16_f32(2 * HALF_M, tl.swap ? tl.ntok : 2 * HALF_M);
@@ -517,7 +561,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const int acc = eg;
         AccSchedule sched;
         __nv_bfloat16* out = g.out;
-        for (int tile = cluster; tile < total; tile += n_clusters) {
+        for (int qi = 0;; ++qi) {
+            const int slot = qi % TQ;
+            if (!mbar_wait_cluster(&tq_full[slot], (qi / TQ) & 1, g.wait_ns, abort_flag, g.status)) break;
+            const int tile = tq[slot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tq_empty[slot]), 0));
+            if (tile >= total) break;
             const Tile tl = decode(tile);
             if (!((sched.buffers(tl.wide) >> acc) & 1)) {
                 sched.advance(tl.wide);
@@ -727,6 +777,7 @@ cudaError_t launch_pair(const CUtensorMap& mr, const CUtensorMap& mw, const CUte
         while (a.stages > 2 && Layout<MODE>(a.stages).bytes(a.n_groups) > static_cast<size_t>(max_optin[dev])) --a.stages;
     const size_t smem = Layout<MODE>(a.stages).bytes(a.n_groups);
     if (smem > static_cast<size_t>(max_optin[dev])) return cudaErrorInvalidValue;
+    if ((e = cudaMemsetAsync(a.tile_ctr, 0, sizeof(int), st)) != cudaSuccess) return e;
     umma_pair_kernel<MODE, F8><<<grid, NUM_THREADS, smem, st>>>(mr, mw, mt, a);
     return cudaGetLastError();
 }
@@ -757,6 +808,7 @@ PairArgs swiglu_args(int64_t rows_cap, const int32_t* offsets, int N, int d, int
     a.status = status;
     a.wait_ns = wait_limit_ns();
     a.clock_probe = clock_probe();
+    a.tile_ctr = reinterpret_cast<int*>(status + 16);
     a.abort_kstep = debug_abort_kstep();
     a.rows_cap = rows_cap;
     a.ldo = I;
@@ -818,6 +870,7 @@ PairArgs down_args(int64_t rows_cap, const int32_t* offsets, int N, int d, int I
     a.status = status;
     a.wait_ns = wait_limit_ns();
     a.clock_probe = clock_probe() ? clock_probe() + 4 : nullptr;
+    a.tile_ctr = reinterpret_cast<int*>(status + 32);
     a.abort_kstep = debug_abort_kstep();
     a.rows_cap = rows_cap;
     a.ldo = d;
