@@ -47,8 +47,9 @@
 // it runs floor(c_e / 256) row tiles, and its leftover rows run as one more row tile if there are
 // at least rem_rows of them, else as weight tiles (N rounded up to 64). GEMM 1: cold_rows =
 // rem_rows = 128; GEMM 2: cold_rows = rem_rows = 256. The tile list (built on the device from
-// offsets, identically by every CTA) is: for each hot expert in order, its row tiles then its
-// leftover weight tiles; then the weight tiles of every cold expert.
+// offsets, identically by every CTA) is: for each hot expert in order, its row tiles (every row
+// block of its first slice of output features, then of the next slice, ...) then its leftover
+// weight tiles; then the weight tiles of every cold expert.
 // Tiles are handed out in list order as pairs become free: the leader's producer takes the next
 // tile index from a counter in global memory (zeroed before each launch) when it starts a tile,
 // and passes it to every role of both CTAs through a queue of TQ tile indices in shared memory
@@ -357,12 +358,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             tl.grp = e;
             tl.dbl = 0;
             if (local < nrow) {
-                const int mt = local / g.ntiles;
+                // feature-major: every row block of one slice of output features, then the next
+                // slice, so the tiles that read the same weight slice are handed out together
+                const int nblk = nrow / g.ntiles;
+                const int mt = local % nblk;
+                const int nt = local / nblk;
                 tl.swap = 0;
                 tl.wide = g.wide;
                 tl.row0 = static_cast<int64_t>(__ldg(offs + (e))) + static_cast<int64_t>(mt) * 2 * HALF_M;
                 tl.rows = min(2 * HALF_M, cnt - mt * 2 * HALF_M);
-                tl.n0 = (local - mt * g.ntiles) * g.tile_cols * (g.wide ? 2 : 1);
+                tl.n0 = nt * g.tile_cols * (g.wide ? 2 : 1);
                 tl.ntok = 0;
             } else {
                 tl.swap = 1;
