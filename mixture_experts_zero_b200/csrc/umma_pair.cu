@@ -38,7 +38,7 @@
 //     A GEMM 2 weight tile of N <= 128 is "double" (when d is a multiple of 512): it loads two
 //     boxes of weight rows per k-step, 256 output features apart, and issues their MMAs on the
 //     same token rows into columns [0, N) and [128, 128 + N): 512 features per tile, so a stage
-//     carries twice the weight bytes per token byte and the ring keeps 5/3 the weight bytes in
+//     carries twice the weight bytes per token byte and the ring keeps twice the weight bytes in
 //     flight of a plain weight tile (the cold experts' tiles are a weight stream whose rate per
 //     SM is set by the bytes in flight).
 // Accumulators: a wide row tile takes both; every other tile takes the next one in turn, so the
@@ -83,16 +83,16 @@ constexpr int TQ = 8;                       // depth of the tile-index queue
 
 enum Mode : int { MODE_SWIGLU = 1, MODE_DOWN = 2 };
 
-// Shared-memory ring of each GEMM. GEMM 1 stages hold the row box and two weight boxes (a wide
-// row tile's two accumulators, or a weight tile's gate and up rows plus up to 64 token rows): 48 KB
-// in 4 stages. GEMM 2 stages hold two boxes (rows and weights, or weights and up to 128 token
-// rows) or a double weight tile's two weight boxes and up to 64 token rows: 40 KB in 5 stages.
-// `stages` is the depth when the per-expert tables fit beside it; launch_pair takes one stage
-// fewer at a time until they do (very many experts).
+// Shared-memory ring, the same for both GEMMs: a stage holds the row box and two weight boxes (a
+// wide row tile's two accumulators), a GEMM 1 weight tile's gate and up rows plus up to 64 token
+// rows, a GEMM 2 double weight tile's two weight boxes plus up to 64 token rows, or a plain
+// weight tile's box plus up to 128 token rows: 48 KB in 4 stages. `stages` is the depth when the
+// per-expert tables fit beside it; for GEMM 2 launch_pair takes one stage fewer at a time until
+// they do (very many experts).
 template <int MODE>
 struct Ring {
-    static constexpr int stages = MODE == MODE_DOWN ? 5 : 4;
-    static constexpr int bytes = MODE == MODE_DOWN ? 2 * A_BYTES + 64 * BK * 2 : 3 * A_BYTES;
+    static constexpr int stages = 4;
+    static constexpr int bytes = 3 * A_BYTES;
 };
 
 struct PairArgs {
@@ -758,8 +758,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 template <int MODE, bool F8>
 cudaError_t launch_pair(const CUtensorMap& mr, const CUtensorMap& mw, const CUtensorMap& mt,
                         const PairArgs& args, int grid, cudaStream_t st) {
-    // a GEMM 2 stage holds two boxes: its row tiles are never wide
-    if (MODE == MODE_DOWN && args.wide) return cudaErrorInvalidValue;
     if (MODE == MODE_SWIGLU && args.dbl) return cudaErrorInvalidValue;
     // once per device: allow the kernel the device's whole opt-in shared memory
     static PerDeviceOnce setup;
@@ -882,12 +880,11 @@ PairArgs down_args(int64_t rows_cap, const int32_t* offsets, int N, int d, int I
     a.n_groups = N;
     a.kdim = I;
     a.n_out = d;
-    // 256 output features per accumulator. Wide row tiles (512 features) measured slower here:
-    // with K = I the main loop of a tile is short, and the unoverlapped epilogue of a wide tile
-    // costs more than the row-operand bytes it saves
+    // 256 output features per accumulator; wide row tiles (512 features, both accumulators) when
+    // d is a multiple of 512
     a.tile_cols = 2 * HALF_M;
-    a.wide = 0;
-    a.ntiles = (d + 2 * HALF_M - 1) / (2 * HALF_M);
+    a.wide = d % (4 * HALF_M) == 0 ? 1 : 0;
+    a.ntiles = a.wide ? d / (4 * HALF_M) : (d + 2 * HALF_M - 1) / (2 * HALF_M);
     a.b_group_rows = d;
     a.up_off = 0;
     a.s_tiles = (d + 2 * HALF_M - 1) / (2 * HALF_M);
