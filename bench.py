@@ -167,13 +167,13 @@ def gemm_phase_roofline(counts, d: int, I: int, f8: bool, mhz: dict, sm_count: i
     work at the SM clock measured inside the kernel (8192 bf16 / 16384 E4M3 FLOP per SM per
     cycle), the other rows' experts (cold experts, and the leftover rows of hot ones) are weight
     streams at the measured copy bandwidth; the bound runs the two kinds one after the other.
-    GEMM 1 (gate/up): row tiles from 128 rows (a 128..255-row remainder included); GEMM 2: from
-    256. counts: rows per FFN expert."""
+    Both GEMMs take row tiles from 128 rows (a 128..255-row remainder included). counts: rows
+    per FFN expert."""
     out = {}
     wb = 1 if f8 else 2
     for name, cold, rem_rows, fl_per_row, w_bytes in (
             ("gemm1_swiglu", 128, 128, 4.0 * d * I, 2 * I * d * wb),
-            ("gemm2_down", 256, 256, 2.0 * d * I, d * I * wb)):
+            ("gemm2_down", 128, 128, 2.0 * d * I, d * I * wb)):
         if not mhz.get(name):
             continue
         hot_rows = 0

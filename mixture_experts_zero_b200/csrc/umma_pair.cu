@@ -33,8 +33,9 @@
 //     columns instead of once per 256, a quarter fewer bytes from L2 per FLOP. Its two halves
 //     are drained by the two epilogue groups in parallel.
 //   weight tiles ("swap"): 256 weight rows (128 per CTA) on the M side and the rows of one expert,
-//     rounded up to 64 and split between the CTAs, on the N side (N <= 128 for GEMM 1, <= 256 for
-//     GEMM 2). GEMM 1 issues a gate MMA into columns [0, N) and an up MMA into [128, 128 + N).
+//     rounded up to 64 and split between the CTAs, on the N side (N <= 128; the kernel handles
+//     N up to 256 in GEMM 2 should rem_rows be raised). GEMM 1 issues a gate MMA into columns
+//     [0, N) and an up MMA into [128, 128 + N).
 //     A GEMM 2 weight tile of N <= 128 is "double" (when d is a multiple of 512): it loads two
 //     boxes of weight rows per k-step, 256 output features apart, and issues their MMAs on the
 //     same token rows into columns [0, N) and [128, 128 + N): 512 features per tile, so a stage
@@ -45,8 +46,9 @@
 // epilogue of one weight tile or narrow row tile overlaps the main loop of the next.
 // Per expert with c_e rows: below cold_rows it is "cold" and runs as weight tiles only; otherwise
 // it runs floor(c_e / 256) row tiles, and its leftover rows run as one more row tile if there are
-// at least rem_rows of them, else as weight tiles (N rounded up to 64). GEMM 1: cold_rows =
-// rem_rows = 128; GEMM 2: cold_rows = rem_rows = 256. The tile list (built on the device from
+// at least rem_rows of them, else as weight tiles (N rounded up to 64). Both GEMMs: cold_rows =
+// rem_rows = 128, so every weight tile has N <= 128 (a GEMM 2 weight tile is then double when d
+// is a multiple of 512). The tile list (built on the device from
 // offsets, identically by every CTA) is: for each hot expert in order, its row tiles (every row
 // block of its first slice of output features, then of the next slice, ...) then its leftover
 // weight tiles; then the weight tiles of every cold expert.
@@ -888,8 +890,8 @@ PairArgs down_args(int64_t rows_cap, const int32_t* offsets, int N, int d, int I
     a.b_group_rows = d;
     a.up_off = 0;
     a.s_tiles = (d + 2 * HALF_M - 1) / (2 * HALF_M);
-    a.cold_rows = 256;
-    a.rem_rows = 256;
+    a.cold_rows = 128;
+    a.rem_rows = 128;
     a.dbl = d % (4 * HALF_M) == 0 ? 1 : 0;
     return a;
 }

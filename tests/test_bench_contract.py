@@ -106,9 +106,9 @@ def test_control_loop_cpu_baseline_times_route_and_update():
 
 
 def test_gemm_phase_roofline_splits_rows_by_tile_kind():
-    """Rows per expert 0, 100, 200, 300 and 600: GEMM 1 takes rows into 256-row tiles from 128 rows
-    (200; 256 of 300 with a 44-row leftover streamed; 512 of 600 with an 88-row leftover streamed)
-    and streams the 100-row expert's weights; GEMM 2 starts row tiles at 256 rows."""
+    """Rows per expert 0, 100, 200, 300 and 600: both GEMMs take rows into 256-row tiles from 128
+    rows (200; 256 of 300 with a 44-row leftover streamed; 512 of 600 with an 88-row leftover
+    streamed) and stream the 100-row expert's weights."""
     sys.path.insert(0, str(ROOT))
     import bench
     d, I = 64, 32
@@ -118,11 +118,11 @@ def test_gemm_phase_roofline_splits_rows_by_tile_kind():
     g1, g2 = r["gemm1_swiglu"], r["gemm2_down"]
     assert g1["rows_in_row_tiles"] == 200 + 256 + 512
     assert g1["weight_stream_bytes"] == 3 * (2 * I * d * 2)  # the 100-row expert and two leftovers
-    assert g2["rows_in_row_tiles"] == 256 + 512
-    assert g2["weight_stream_bytes"] == 4 * (d * I * 2)      # 100, 200 and the two leftovers
+    assert g2["rows_in_row_tiles"] == 200 + 256 + 512
+    assert g2["weight_stream_bytes"] == 3 * (d * I * 2)      # the 100-row expert and two leftovers
     rate = 2 * 8192 * 1000.0e6
     assert abs(g1["tensor_ms"] - 1e3 * 4.0 * d * I * 968 / rate) < 1e-3
-    assert abs(g2["stream_ms"] - 1e3 * 4 * d * I * 2 / 1e9) < 1e-3
+    assert abs(g2["stream_ms"] - 1e3 * 3 * d * I * 2 / 1e9) < 1e-3
     assert g1["frac"] == round(g1["t_bound_ms"] / 1.0, 4)
     # no clock measured for a GEMM: no entry
     assert bench.gemm_phase_roofline(counts, d, I, False, {"gemm1_swiglu": None}, 2, 1.0, {}) == {}

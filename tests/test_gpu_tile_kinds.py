@@ -6,10 +6,9 @@ work) split each expert's rows into tiles by its row count c:
   GEMM 1 (gate/up + SwiGLU): c < 128: weight tiles only ("cold"); otherwise floor(c/256) full
     256-row tiles, a remainder of 128..255 rows as one more (padded) row tile, and a remainder
     below 128 rows as leftover weight tiles;
-  GEMM 2 (down): c < 256: weight tiles only, their token width rounded up to 64 (up to 256
-    columns, so cold experts with 129..255 rows take the 192/256-wide form, and those with at most
-    128 rows the double form of 512 output features per tile); otherwise full 256-row tiles and
-    the remainder as leftover weight tiles (double when the remainder is at most 128 rows).
+  GEMM 2 (down): the same row rules as GEMM 1 (weight tiles below 128 rows, a padded
+    128..255-row remainder tile, leftover weight tiles below 128 rows); its weight tiles take the
+    double form of 512 output features per tile (d is a multiple of 512 here).
 The rules are restated here from that description, independently of the kernel, to pick rows: for
 each kind, the first and the last row of one tile of that kind (every output column of those rows
 is checked, so every feature tile of both accumulators is covered). The test fails if the
@@ -52,22 +51,23 @@ def tile_rows(off: np.ndarray):
             elif rem > 0:
                 note((1, "leftover weight tile"), e, o + nfull * 256, o + c - 1)
         # GEMM 2
-        if c < 256:
-            kind = "cold weight tile, N > 128" if (c + 63) // 64 * 64 > 128 else "cold double weight tile"
-            note((2, kind), e, o, o + c - 1)
+        if c < 128:
+            note((2, "cold double weight tile"), e, o, o + c - 1)
         else:
             nfull, rem = divmod(c, 256)
-            note((2, "full 256-row tile"), e, o, o + 255)
-            if rem:
-                kind = "leftover weight tile, N > 128" if rem > 128 else "leftover double weight tile"
-                note((2, kind), e, o + nfull * 256, o + c - 1)
+            if nfull:
+                note((2, "full 256-row tile"), e, o, o + 255)
+            if rem >= 128:
+                note((2, "padded 128..255-row remainder tile"), e, o + nfull * 256, o + c - 1)
+            elif rem > 0:
+                note((2, "leftover double weight tile"), e, o + nfull * 256, o + c - 1)
     return found
 
 
 KINDS = {(1, "cold weight tile"), (1, "full 256-row tile"), (1, "full 256-row tile, last block"),
          (1, "padded 128..255-row remainder tile"), (1, "leftover weight tile"),
-         (2, "cold weight tile, N > 128"), (2, "cold double weight tile"),
-         (2, "full 256-row tile"), (2, "leftover weight tile, N > 128"), (2, "leftover double weight tile")}
+         (2, "cold double weight tile"), (2, "full 256-row tile"),
+         (2, "padded 128..255-row remainder tile"), (2, "leftover double weight tile")}
 
 
 def _selected_rows(off):
