@@ -33,7 +33,7 @@
 //     columns instead of once per 256, a quarter fewer bytes from L2 per FLOP. Its two halves
 //     are drained by the two epilogue groups in parallel.
 //   weight tiles ("swap"): 256 weight rows (128 per CTA) on the M side and the rows of one expert,
-//     rounded up to 32 and split between the CTAs, on the N side (N <= 128; the kernel handles
+//     rounded up to 16 and split between the CTAs, on the N side (N <= 128; the kernel handles
 //     N up to 256 in GEMM 2 should rem_rows be raised). GEMM 1 issues a gate MMA into columns
 //     [0, N) and an up MMA into [128, 128 + N).
 //     A GEMM 2 weight tile of N <= 128 is "double" (when d is a multiple of 512): it loads two
@@ -46,7 +46,7 @@
 // epilogue of one weight tile or narrow row tile overlaps the main loop of the next.
 // Per expert with c_e rows: below cold_rows it is "cold" and runs as weight tiles only; otherwise
 // it runs floor(c_e / 256) row tiles, and its leftover rows run as one more row tile if there are
-// at least rem_rows of them, else as weight tiles (N rounded up to 32). Both GEMMs: cold_rows =
+// at least rem_rows of them, else as weight tiles (N rounded up to 16). Both GEMMs: cold_rows =
 // rem_rows = 128, so every weight tile has N <= 128 (a GEMM 2 weight tile is then double when d
 // is a multiple of 512). The tile list (built on the device from
 // offsets, identically by every CTA) is: for each hot expert in order, its row tiles (every row
@@ -79,7 +79,7 @@ constexpr int A_BYTES = HALF_M * BK * 2;    // 16 KB: one 128-row operand box of
 constexpr int TMEM_COLS = 512;
 constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;              // warps 4..11: two epilogue groups of four warps
-constexpr int TOK_BOX = 16;                 // token rows per TMA box of a weight tile (per CTA)
+constexpr int TOK_BOX = 8;                  // token rows per TMA box of a weight tile (per CTA)
 constexpr int TOK_ROUND = 2 * TOK_BOX;      // weight-tile N is a multiple of this
 constexpr int TQ = 8;                       // depth of the tile-index queue
 
