@@ -126,3 +126,19 @@ def test_gemm_phase_roofline_splits_rows_by_tile_kind():
     assert g1["frac"] == round(g1["t_bound_ms"] / 1.0, 4)
     # no clock measured for a GEMM: no entry
     assert bench.gemm_phase_roofline(counts, d, I, False, {"gemm1_swiglu": None}, 2, 1.0, {}) == {}
+
+
+def test_clock_summary_reports_load_clock_reasons_and_power_limit():
+    """The `clocks` block: the median SM clock of the samples under load (power above half the
+    largest sample), the throttle reasons seen active, and the enforced power limit."""
+    sys.path.insert(0, str(ROOT))
+    import bench
+    rows = [["t", "GPU-x", "1965", "1965", "120.0", "0x0", "Not Active", "Not Active", "Not Active", "Not Active", "1000.00"],
+            ["t", "GPU-x", "1300", "1965", "990.0", "0x4", "Not Active", "Not Active", "Not Active", "Active", "1000.00"],
+            ["t", "GPU-x", "1400", "1965", "960.0", "0x4", "Not Active", "Not Active", "Not Active", "Active", "1000.00"]]
+    c = bench.ClockSampler.summarize(rows)
+    assert c["sm_mhz"] == 1350.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"] and c["power_limit_w"] == 1000.0
+    assert c["samples"] == 3 and c["samples_under_load"] == 2
+    # no sampler output: the block says so instead of inventing a clock
+    assert bench.ClockSampler.summarize([])["reasons"] == ["nvidia-smi unavailable"]
