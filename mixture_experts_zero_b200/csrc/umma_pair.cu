@@ -48,13 +48,14 @@
 // it runs floor(c_e / 256) row tiles, and its leftover rows run as one more row tile if there are
 // at least rem_rows of them, else as weight tiles (N rounded up to 16). Both GEMMs: cold_rows =
 // rem_rows = 128, so every weight tile has N <= 128 (a GEMM 2 weight tile is then double when d
-// is a multiple of 512). The tile list (built on the device from
-// offsets, identically by every CTA) is: for each hot expert in order, its row tiles (every row
-// block of its first slice of output features, then of the next slice, ...) then its leftover
-// weight tiles; then the weight tiles of every cold expert.
-// Tiles are handed out in list order as pairs become free: the leader's producer takes the next
-// tile index from a counter in global memory (zeroed before each launch) when it starts a tile,
-// and passes it to every role of both CTAs through a queue of TQ tile indices in shared memory
+// is a multiple of 512). The tile list (built on the device from offsets, identically by every
+// CTA) is: for each hot expert in order, its row tiles (every row block of its first slice of
+// output features, then of the next slice, ...) then its leftover weight tiles; then the weight
+// tiles of every cold expert.
+// Tiles are handed out in list order as pairs become free: as the leader's producer starts a
+// tile it takes the index of its next one from a counter in global memory (zeroed before each
+// launch), and it passes each index to every role of both CTAs through a queue of TQ tile
+// indices in shared memory
 // (a full barrier per slot in each CTA, released by the leader's producer; an empty barrier per
 // slot in the leader, which counts the 18 other readers: the MMA issuer, the eight epilogue warps
 // of each CTA and the peer's producer). The tiles that share a hot expert's weights then start
