@@ -121,3 +121,14 @@ def test_the_cuda_package_never_imports_the_oracle():
         text = f.read_text()
         assert "import oracle" not in text and "from oracle" not in text, f
         assert "moe_oracle" not in text, f
+
+
+def test_clock_probe_setting_needs_no_device_and_checks_its_buffer(lib):
+    """The probe is a process-wide pointer the library stores (no CUDA call): setting and clearing
+    it works without a GPU, and the binding refuses a buffer that is not 8 int64 on the device."""
+    import torch
+    binding.lc_moe_set_clock_probe(None)
+    with pytest.raises(AssertionError):
+        binding.lc_moe_set_clock_probe(torch.zeros(8, dtype=torch.int64))  # host memory
+    lib.lc_moe_set_clock_probe(ctypes.c_void_p(0x1000))
+    lib.lc_moe_set_clock_probe(None)
